@@ -1,0 +1,381 @@
+"""Benchmark of the paged MLA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3] [--impl reference]
+
+One step = one pass of the whole hot path over one batch: the split-KV scheduler
+(mla_get_metadata), the split kernel and the LSE combine (mla_decode_fwd), all through
+the C ABI. The default workload is DeepSeek-V3-shaped decode: batch 128, s_q 1, 128
+query heads, one shared 576-dim latent head, lengths uniform in [1, 8192], 64-token
+bf16 pages randomly permuted in the pool. Inputs are seeded synthetic data.
+
+Rank 0 prints one JSON line. `value` is algorithmic HBM bytes (every visible KV row
+once, q, out, lse) of all ranks' steps divided by the max-over-ranks device time;
+`roofline` relates the decode call to the measured peaks; `e2e` repeats the measurement
+with q, block table and lengths copied from pinned host memory and the outputs read
+back every step; `cpu_baseline` times the fp64 CPU oracle on a bounded sample.
+With N > 1 each rank decodes its own batch (weak scaling, no data-path collective).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_paged_kv_06_b200 import workloads as wl  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
+LAUNCHES_PER_STEP = 3               # metadata, split kernel, combine kernel
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="v3", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def metric_name():
+    return "MLA decode HBM GB/s, TFLOPS and μs/call at b=128,h_q=128; fraction of roofline"
+
+
+def workload_config(x, name):
+    w = wl.WORKLOADS[name]
+    return {"workload": f"{name}: {w.description}", "batch": x.batch, "s_q": x.s_q,
+            "h_q": x.h_q, "d": 576, "dv": 512, "block_size": 64, "causal": bool(x.causal),
+            "num_blocks": x.num_blocks, "total_tokens": int(x.seqlens.sum()),
+            "seed": x.seed}
+
+
+# ---------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        if not getattr(self, "lines", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [c.strip() for c in ln.split(",")]
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        loaded = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------
+def cpu_baseline(x, seconds):
+    """Time the fp64 oracle on a bounded sample of the workload's sequences."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+    order = sorted(range(x.batch), key=lambda b: int(x.seqlens[b]))
+    picked, spent, nbytes = [], 0.0, 0
+    g = torch.Generator().manual_seed(123)
+    perm = torch.randperm(x.batch, generator=g).tolist()
+    for b in perm:
+        t0 = time.perf_counter()
+        oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale, x.causal,
+                      batch_indices=[b])
+        spent += time.perf_counter() - t0
+        picked.append(b)
+        nbytes += wl.algorithmic_work(x.seqlens[b:b + 1], x.s_q, x.h_q, x.causal)[0]
+        if spent >= seconds:
+            break
+    del order
+    return {"value": nbytes / spent / 1e9, "unit": "GB/s", "cores": int(cores),
+            "kind": "oracle",
+            "sample": f"{len(picked)} of {x.batch} sequences of the same workload "
+                      f"({sum(int(x.seqlens[b]) for b in picked)} tokens), one oracle.decode "
+                      f"call each, {spent:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, timed on the host cores, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    x = wl.make_workload(args.workload, seed=args.seed)
+    g = torch.Generator().manual_seed(99)
+    perm = torch.randperm(x.batch, generator=g).tolist()
+    per_step = 2                       # sequences per step: a bounded sample
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+
+    def step(k):
+        bs = [perm[(k * per_step + j) % x.batch] for j in range(per_step)]
+        oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale, x.causal,
+                      batch_indices=bs)
+        return sum(wl.algorithmic_work(x.seqlens[b:b + 1], x.s_q, x.h_q, x.causal)[0]
+                   for b in bs)
+
+    for k in range(args.warmup):
+        step(k)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for k in range(args.steps):
+        nbytes += step(args.warmup + k)
+    dt = time.perf_counter() - t0
+    val = nbytes / dt / 1e9
+    line = {"metric": metric_name(), "value": val, "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(x, args.workload),
+            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": int(cores),
+                             "kind": "oracle",
+                             "sample": f"{per_step} sequences per step of the same workload"},
+            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    from mla_paged_kv_06_b200 import mla
+
+    # each rank decodes its own batch of the same shape (weak scaling)
+    x = wl.make_workload(args.workload, seed=args.seed + rank)
+    d = dict(q=x.q.cuda(), kcache=x.kcache.cuda(), block_table=x.block_table.cuda(),
+             seqlens=x.seqlens.cuda())
+    nsm = mla.default_num_sms()
+    meta = torch.empty(mla.mla_metadata_ints(nsm), dtype=torch.int32, device="cuda")
+    ns = torch.empty(mla.mla_num_splits_len(x.batch, x.h_q, x.s_q), dtype=torch.int32,
+                     device="cuda")
+    ws = torch.empty(mla.mla_workspace_bytes(x.batch, x.h_q, x.s_q, nsm), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((x.batch, x.s_q, x.h_q, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    nbytes, nflops = wl.algorithmic_work(x.seqlens, x.s_q, x.h_q, x.causal)
+
+    def step():
+        mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
+        mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
+                           x.causal, meta, ns, ws, out, lse)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, word = mla.mla_get_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error during warm-up: {mla.status_string(st)} {word:#x}")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            flush.zero_()                                  # untimed L2 flush
+            e0, e1, e2 = ev[k]
+            e0.record(stream)
+            mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
+            e1.record(stream)
+            mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
+                               x.causal, meta, ns, ws, out, lse)
+            e2.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
+    decode_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    meta_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st, word = mla.mla_get_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error during timing: {mla.status_string(st)} {word:#x}")
+
+    # end to end through the public call with host buffers: q, block table and lengths
+    # copied in from pinned memory and out + lse read back every step
+    hq = x.q.pin_memory()
+    hbt = x.block_table.pin_memory()
+    hsl = x.seqlens.pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = hq.numel() * 2 + hbt.numel() * 4 + hsl.numel() * 4
+    d2h = hout.numel() * 2 + hlse.numel() * 4
+
+    def e2e_step():
+        d["q"].copy_(hq, non_blocking=True)
+        d["block_table"].copy_(hbt, non_blocking=True)
+        d["seqlens"].copy_(hsl, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = 0.0
+    for k in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms += a.elapsed_time(b)
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    hbm_peak, tf_peak, peak_kind = peaks()
+    avg_decode_s = statistics.mean(decode_ms) / 1e3
+    achieved_gbs = nbytes / avg_decode_s / 1e9
+    achieved_tf = nflops / avg_decode_s / 1e12
+    t_bytes = nbytes / (hbm_peak * 1e9)
+    t_flops = nflops / (tf_peak * 1e12)
+    bound = "hbm" if t_bytes >= t_flops else "tensor"
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        try:
+            with open(prof) as f:
+                tj = json.load(f)
+            if tj.get("workload") == args.workload and tj.get("kernel_rev") == KERNEL_REV:
+                traffic = tj.get("bytes_per_launch")
+        except Exception:
+            traffic = None
+    roof = {"bound": bound, "kernel": "mla_decode_fwd (split kernel + combine kernel)",
+            "achieved": achieved_gbs if bound == "hbm" else achieved_tf,
+            "peak": hbm_peak if bound == "hbm" else tf_peak,
+            "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured"
+            else "fallback",
+            "frac": (achieved_gbs / hbm_peak) if bound == "hbm" else (achieved_tf / tf_peak),
+            "traffic": traffic,
+            "hbm_frac": achieved_gbs / hbm_peak, "tensor_frac": achieved_tf / tf_peak,
+            "roofline_frac": max(t_bytes, t_flops) / avg_decode_s,
+            "algorithmic_bytes": nbytes, "algorithmic_flops": nflops}
+
+    value = nbytes * args.steps * world / (total_ms / 1e3) / 1e9
+    line = {"metric": metric_name(), "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 q and cache; seeded lengths and page permutation)",
+            "config": dict(workload_config(x, args.workload),
+                           l2="L2 flushed (256 MB write, untimed) before every step; the step's "
+                              "KV rows exceed L2", parallelism=f"replicas x{world}"),
+            "tflops": nflops * args.steps * world / (total_ms / 1e3) / 1e12,
+            "us_per_call": statistics.median(step_ms) * 1e3,
+            "us_per_call_decode": statistics.median(decode_ms) * 1e3,
+            "us_per_call_metadata": statistics.median(meta_ms) * 1e3,
+            "roofline": roof,
+            "e2e": {"value": nbytes * args.steps * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "note": "KV cache resident in HBM as decode state; per-step inputs are "
+                            "q, block table and lengths"},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+# Bumped whenever the split kernel changes, so stale ncu traffic is never reported.
+KERNEL_REV = "simt-1"
+
+if __name__ == "__main__":
+    sys.exit(main())

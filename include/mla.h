@@ -1,0 +1,185 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) paged MLA decode library (libmla_b200.so).
+ *
+ * Operation (Multi-head Latent Attention decode over a paged latent cache; the
+ * FlashMLA release article «DeepSeek open-sources FlashMLA», shoujike.com.cn,
+ * paragraphs on the MLA decode kernel for variable-length sequences, on the paged
+ * BF16 kvcache with block size 64 and on compressing keys and values into one latent
+ * vector per token):
+ *
+ *   every query row r = (i, h) of sequence b attends to the visible tokens t < n_i of
+ *   that sequence, n_i = L_b - s_q + i + 1 when causal, else L_b;
+ *   K_t is the token's 576-dim latent cache row (512 latent + 64 rope dims), shared by
+ *   all heads, and V_t is its first 512 dims;
+ *     s_t    = scale * <q[b,i,h,:], K_t>
+ *     out    = sum_t softmax(s)_t * V_t            (bf16, round-to-nearest-even)
+ *     lse    = ln sum_t exp(s_t)                   (fp32, natural log)
+ *   A row with no visible token gets out = 0 and lse = -inf.
+ *
+ * Data layout (all tensors dense, row-major, caller-owned device memory):
+ *   q            bf16  [batch][s_q][h_q][576]
+ *   kcache       bf16  [num_blocks][64][1][576]      pool of 64-token pages
+ *   block_table  int32 [batch][max_blocks]           physical page of logical page j
+ *   seqlens      int32 [batch]                       0 <= L_b <= 64 * max_blocks
+ *   out          bf16  [batch][s_q][h_q][512]
+ *   lse          fp32  [batch][h_q][s_q]
+ * Query rows are numbered r = i * h_q + h and cut into tiles of 128 rows; a
+ * "work sequence" is one (tile, sequence) pair, v = tile * batch + b.
+ *
+ * Ownership: the library allocates nothing on these calls. The caller owns every
+ * buffer, including `metadata`, `num_splits` and `workspace`, and must keep them alive
+ * until the stream work that uses them has finished.
+ *
+ * Asynchrony: mla_get_metadata and mla_decode_fwd only enqueue work on `stream`
+ * (a cudaStream_t passed as void*; NULL is the legacy default stream) and never
+ * synchronise, so both can be captured in a CUDA graph.
+ *
+ * Errors: every call checks its arguments on the host first and returns a negative
+ * mla_status without launching anything when they are invalid. A launch failure is
+ * MLA_ERR_CUDA. Problems only the device can see (a sequence longer than its block
+ * table, a block id outside the pool, a pipeline wait that ran out of its iteration
+ * limit) never trap: the kernel skips the offending access, records a code in a
+ * device-side error word and finishes; mla_get_last_device_error reports and clears
+ * it. Outputs of a call that recorded an error are unspecified.
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every declaration below is exported from libmla_b200.so (built with hidden default
+ * visibility). */
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef int mla_status;
+
+#define MLA_OK                        0
+#define MLA_ERR_INVALID_ARG          -1  /* null pointer, bad size, misaligned buffer   */
+#define MLA_ERR_UNSUPPORTED          -2  /* shape outside the supported set             */
+#define MLA_ERR_CUDA                 -3  /* a CUDA runtime/driver call failed           */
+#define MLA_ERR_WORKSPACE_TOO_SMALL  -4  /* workspace_bytes < mla_workspace_bytes(...)  */
+#define MLA_ERR_DEVICE_TIMEOUT       -5  /* a bounded pipeline wait gave up             */
+#define MLA_ERR_DEVICE_BAD_INPUT     -6  /* seqlen > 64*max_blocks or block id >= pool  */
+
+#define MLA_HEAD_DIM        576   /* latent (512) + rope (64) dims per cache row      */
+#define MLA_HEAD_DIM_V      512   /* V = first 512 dims of the row                    */
+#define MLA_BLOCK_SIZE       64   /* tokens per page                                  */
+#define MLA_TILE_ROWS       128   /* query rows per work tile                         */
+#define MLA_MAX_H_Q         128
+#define MLA_MAX_S_Q          16
+#define MLA_MAX_ROWS       1024   /* s_q * h_q                                        */
+#define MLA_MAX_BATCH     65536
+#define MLA_METADATA_INTS_PER_UNIT 8
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* mla_status_string(mla_status status);
+
+/* Number of int32 entries `metadata` must hold for a given num_sms (>= 1):
+ * 8 * (num_sms + 1). */
+size_t mla_metadata_ints(int num_sms);
+
+/* Number of int32 entries `num_splits` must hold: batch * ceil(s_q*h_q/128) + 1. */
+size_t mla_num_splits_len(int batch, int h_q, int s_q);
+
+/* Bytes of `workspace` mla_decode_fwd needs for these sizes (fp32 split partials:
+ * one [128][512] output tile and one [128] lse tile per possible split). Returns 0
+ * for sizes the library rejects. */
+size_t mla_workspace_bytes(int batch, int h_q, int s_q, int num_sms);
+
+/* Work units (pairs of SMs) a schedule for `num_sms` uses on the current device:
+ * min(num_sms / 2, co-resident 2-CTA clusters of the decode kernel), at least 1.
+ * Returns a negative mla_status on failure. */
+int mla_num_work_units(int num_sms);
+
+/*
+ * Split-KV tile scheduler (variable-length batches: FlashMLA release article,
+ * paragraph on dynamic sequence handling). Balances the pages of all work sequences
+ * over the work units: every page of every work sequence is owned by exactly one
+ * unit, each unit owns one contiguous run of pages in (v, page) order, and a work
+ * sequence whose pages span k units is split into k chunks merged by the combine
+ * step of mla_decode_fwd.
+ *
+ *   seqlens     device int32 [batch]
+ *   num_sms     SMs the decode may use (>= 1); 148 on a B200. num_sms = 1 forces a
+ *               single unit and so no splits.
+ *   metadata    device int32 [mla_metadata_ints(num_sms)], written:
+ *               [0..7]   header {num_units, tiles, batch, h_q, s_q, unit_cost, 0, 0}
+ *               [8u+8..] unit u {v_begin, page_begin, v_end, page_end, chunk_begin,0,0,0}
+ *                        (half-open range of (v, page) positions)
+ *   num_splits  device int32 [mla_num_splits_len(batch, h_q, s_q)], written: the
+ *               exclusive prefix sum over work sequences of their chunk counts, so
+ *               chunks of v are num_splits[v] .. num_splits[v+1]-1.
+ * The result depends only on (seqlens, batch, h_q, s_q, num_sms) and the device.
+ */
+mla_status mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q, int num_sms,
+                            int32_t* metadata, int32_t* num_splits, void* stream);
+
+/*
+ * Decode attention (see the operation above). Runs the sm_100a split kernel
+ * (TMA page gather -> tcgen05 QK^T and PV with TMEM accumulators -> fp32 online
+ * softmax with tail and causal masks) and then the LSE-weighted combine kernel.
+ *
+ *   q, kcache, block_table, seqlens, out, lse: device buffers in the layout above;
+ *     q, kcache and out must be 16-byte aligned.
+ *   num_blocks  pages in the pool (>= 1); max_blocks  columns of block_table (>= 1)
+ *   scale       softmax scale applied to q.K (finite)
+ *   causal      0 or 1
+ *   metadata, num_splits  from mla_get_metadata with the same seqlens, batch, h_q, s_q
+ *   workspace   device scratch of workspace_bytes >= mla_workspace_bytes(batch, h_q,
+ *               s_q, num_sms of the metadata call), 256-byte aligned.
+ * Supported: 1 <= h_q <= 128, 1 <= s_q <= 16, s_q*h_q <= 1024, 1 <= batch <= 65536.
+ */
+mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                          const int32_t* block_table, int max_blocks,
+                          const int32_t* seqlens, int batch, int s_q, int h_q,
+                          float scale, int causal,
+                          const int32_t* metadata, const int32_t* num_splits,
+                          void* workspace, size_t workspace_bytes,
+                          uint16_t* out, float* lse, void* stream);
+
+/*
+ * Reads and clears the device-side error word of the current device after
+ * synchronising `stream`. Returns MLA_OK, MLA_ERR_DEVICE_TIMEOUT,
+ * MLA_ERR_DEVICE_BAD_INPUT or MLA_ERR_CUDA. *detail (may be NULL) receives the raw
+ * word: bits 0-7 the error kind, the rest where it arose.
+ */
+mla_status mla_get_last_device_error(void* stream, uint32_t* detail);
+
+/*
+ * Host-side copy of the scheduler, for tests and for callers that plan on the CPU:
+ * the same arithmetic as mla_get_metadata with an explicit unit count, on host
+ * buffers (seqlens_host [batch], metadata_host [8*(num_units+1)],
+ * num_splits_host [mla_num_splits_len]). Needs no GPU.
+ */
+mla_status mla_plan_host(const int32_t* seqlens_host, int batch, int h_q, int s_q,
+                         int num_units, int32_t* metadata_host, int32_t* num_splits_host);
+
+/*
+ * Correctness-first decode on CUDA cores (one warp per query row, no tensor cores).
+ * Same arguments, layouts, metadata and combine as mla_decode_fwd; kept as an
+ * independent second kernel for cross-checking the tensor-core path.
+ */
+mla_status mla_decode_fwd_simt(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                               const int32_t* block_table, int max_blocks,
+                               const int32_t* seqlens, int batch, int s_q, int h_q,
+                               float scale, int causal,
+                               const int32_t* metadata, const int32_t* num_splits,
+                               void* workspace, size_t workspace_bytes,
+                               uint16_t* out, float* lse, void* stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MLA_B200_H_ */

@@ -1,0 +1,115 @@
+// Device split-KV scheduler: one CTA computes the whole schedule so the call needs no
+// host round trip and can sit inside a captured CUDA graph.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+constexpr int kMetaThreads = 1024;
+
+// Block-wide exclusive scan of one int64 per thread; returns the block total.
+__device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* smem_warp,
+                                                        int64_t* out_prefix) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int64_t incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) smem_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int64_t w = lane < (int)(blockDim.x >> 5) ? smem_warp[lane] : 0;
+        int64_t wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int64_t y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        smem_warp[lane] = wi - w;          // exclusive prefix of warp totals
+        if (lane == 31) smem_warp[32] = wi;
+    }
+    __syncthreads();
+    *out_prefix = smem_warp[warp] + incl - x;
+    int64_t total = smem_warp[32];
+    __syncthreads();
+    return total;
+}
+
+// metadata: header {num_units, tiles, batch, h_q, s_q, unit_cost, 0, 0} then one
+// {v_begin, page_begin, v_end, page_end, chunk_begin, 0, 0, 0} per unit.
+// num_splits holds the cumulative costs C[v] while the units are located, then is
+// overwritten with the chunk prefix.
+__global__ void __launch_bounds__(kMetaThreads)
+metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q, int tiles,
+                int num_units,
+                int32_t* __restrict__ metadata, int32_t* __restrict__ num_splits) {
+    __shared__ int64_t warp_sums[33];
+    __shared__ int64_t s_total;
+    const int V = batch * tiles;
+    auto pages = [&](int v) {
+        int L = seqlens[v % batch];
+        return pages_of(L < 0 ? 0 : L);
+    };
+
+    // Phase 1: cumulative costs.
+    int64_t carry = 0;
+    for (int base = 0; base < V; base += blockDim.x) {
+        int v = base + threadIdx.x;
+        int64_t cost = v < V ? (int64_t)kOverheadPages + pages(v) : 0;
+        int64_t pre;
+        int64_t tot = block_exclusive_scan(cost, warp_sums, &pre);
+        int64_t c = carry + pre;
+        if (v < V) {
+            if (c > 0x7fffffffLL) record_error(kErrBadInput, 0xfffffeu);
+            num_splits[v] = (int32_t)(c > 0x7fffffffLL ? 0x7fffffff : c);
+        }
+        carry += tot;
+    }
+    if (threadIdx.x == 0) {
+        if (carry > 0x7fffffffLL) { record_error(kErrBadInput, 0xfffffeu); carry = 0x7fffffff; }
+        num_splits[V] = (int32_t)carry;
+        s_total = carry;
+    }
+    __syncthreads();
+    const int64_t total = s_total;
+    const int64_t W = unit_cost(total, num_units);
+    auto C = [&](int v) { return (int64_t)num_splits[v]; };
+
+    // Phase 2: one thread per unit locates its first and one-past-last page.
+    for (int u = threadIdx.x; u < num_units; u += blockDim.x) {
+        int vb, kb, ve, ke;
+        locate((int64_t)u * W, C, pages, V, kOverheadPages, &vb, &kb);
+        locate((int64_t)(u + 1) * W, C, pages, V, kOverheadPages, &ve, &ke);
+        int chunk = 0;
+        if (vb < V && (vb != ve || kb != ke))
+            chunk = u - unit_of(C(vb) + kOverheadPages, W);
+        int32_t* m = metadata + kMetaInts * (u + 1);
+        m[0] = vb; m[1] = kb; m[2] = ve; m[3] = ke; m[4] = chunk;
+        m[5] = 0; m[6] = 0; m[7] = 0;
+    }
+    if (threadIdx.x == 0) {
+        metadata[0] = num_units; metadata[1] = tiles; metadata[2] = batch;
+        metadata[3] = h_q; metadata[4] = s_q;
+        metadata[5] = (int32_t)(W > 0x7fffffffLL ? 0x7fffffff : W);
+        metadata[6] = 0; metadata[7] = 0;
+    }
+    __syncthreads();
+
+    // Phase 3: chunk counts -> exclusive prefix, written over the costs tile by tile.
+    carry = 0;
+    for (int base = 0; base < V; base += blockDim.x) {
+        int v = base + threadIdx.x;
+        int n = v < V ? chunks_of(C(v), pages(v), W, kOverheadPages) : 0;
+        int64_t pre;
+        int64_t tot = block_exclusive_scan(n, warp_sums, &pre);   // also a barrier
+        if (v < V) num_splits[v] = (int32_t)(carry + pre);
+        carry += tot;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) num_splits[V] = (int32_t)carry;
+}
+
+}  // namespace mla

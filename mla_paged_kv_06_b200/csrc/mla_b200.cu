@@ -1,0 +1,259 @@
+// libmla_b200.so: the C ABI of include/mla.h. This is the library's single translation
+// unit; the kernels live in the headers it includes.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "mla.h"
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "decode_simt.cuh"
+#include "metadata.cuh"
+#include "sched.cuh"
+
+namespace {
+
+using namespace mla;
+
+constexpr size_t kWsHeader = 256;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool shape_ok(int batch, int h_q, int s_q) {
+    return batch >= 1 && batch <= MLA_MAX_BATCH && h_q >= 1 && h_q <= MLA_MAX_H_Q &&
+           s_q >= 1 && s_q <= MLA_MAX_S_Q && h_q * s_q <= MLA_MAX_ROWS;
+}
+
+int units_bound(int num_sms) { return num_sms / 2 < 1 ? 1 : num_sms / 2; }
+
+size_t max_chunks_for(int batch, int h_q, int s_q, int num_sms) {
+    return (size_t)batch * num_tiles(h_q, s_q) + (size_t)units_bound(num_sms);
+}
+
+constexpr size_t kChunkBytes = (size_t)kTileRows * 4 + (size_t)kTileRows * kHeadDimV * 4;
+
+// Partial-slot capacity of a workspace and the byte offset of its output partials.
+size_t ws_capacity(size_t bytes) {
+    if (bytes < kWsHeader + 2 * kAlign) return 0;
+    return (bytes - kWsHeader - 2 * kAlign) / kChunkBytes;
+}
+
+size_t ws_o_offset(size_t cap) { return align_up(kWsHeader + cap * kTileRows * 4, kAlign); }
+
+// SM pairs the decode can keep co-resident on a device (cached per device).
+int device_pairs(int dev) {
+    static std::mutex mu;
+    static std::vector<int> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+    if (cache[dev] > 0) return cache[dev];
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return -1;
+    cache[dev] = sms / 2 < 1 ? 1 : sms / 2;
+    return cache[dev];
+}
+
+mla_status validate_decode(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                           const int32_t* block_table, int max_blocks, const int32_t* seqlens,
+                           int batch, int s_q, int h_q, float scale, int causal,
+                           const int32_t* metadata, const int32_t* num_splits, void* workspace,
+                           size_t workspace_bytes, uint16_t* out, float* lse) {
+    if (!q || !kcache || !block_table || !seqlens || !metadata || !num_splits || !workspace ||
+        !out || !lse)
+        return MLA_ERR_INVALID_ARG;
+    if (num_blocks < 1 || max_blocks < 1 || !std::isfinite(scale) || (causal != 0 && causal != 1))
+        return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)q | (uintptr_t)kcache | (uintptr_t)out) & 15u) return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)workspace) & (kAlign - 1)) return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)lse | (uintptr_t)seqlens | (uintptr_t)block_table) & 3u)
+        return MLA_ERR_INVALID_ARG;
+    if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
+    if ((size_t)num_blocks * kBlock * kHeadDim * 2 >= ((size_t)1 << 47)) return MLA_ERR_UNSUPPORTED;
+    if (workspace_bytes < mla_workspace_bytes(batch, h_q, s_q, 1))
+        return MLA_ERR_WORKSPACE_TOO_SMALL;
+    return MLA_OK;
+}
+
+DecodeParams make_params(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                         const int32_t* block_table, int max_blocks, const int32_t* seqlens,
+                         int batch, int s_q, int h_q, float scale, int causal,
+                         const int32_t* metadata, const int32_t* num_splits, void* workspace,
+                         size_t workspace_bytes, uint16_t* out, float* lse) {
+    DecodeParams p;
+    p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    p.kcache = reinterpret_cast<const __nv_bfloat16*>(kcache);
+    p.block_table = block_table;
+    p.seqlens = seqlens;
+    p.metadata = metadata;
+    p.num_splits = num_splits;
+    const size_t cap = ws_capacity(workspace_bytes);
+    p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeader);
+    p.ws_o = reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_o_offset(cap));
+    p.max_chunks = (int)(cap > 0x7fffffff ? 0x7fffffff : cap);
+    p.out = reinterpret_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.num_blocks = num_blocks;
+    p.max_blocks = max_blocks;
+    p.batch = batch;
+    p.s_q = s_q;
+    p.h_q = h_q;
+    p.rows = s_q * h_q;
+    p.tiles = num_tiles(h_q, s_q);
+    p.scale_log2 = scale * kLog2e;
+    p.causal = causal;
+    return p;
+}
+
+mla_status launch_combine(const DecodeParams& p, cudaStream_t s) {
+    dim3 grid(p.batch * p.tiles, kTileRows / kCombineRowsPerCta);
+    combine_kernel<<<grid, kCombineThreads, 0, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status status) {
+    switch (status) {
+        case MLA_OK: return "MLA_OK";
+        case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+        case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+        case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+        case MLA_ERR_WORKSPACE_TOO_SMALL: return "MLA_ERR_WORKSPACE_TOO_SMALL";
+        case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
+        case MLA_ERR_DEVICE_BAD_INPUT: return "MLA_ERR_DEVICE_BAD_INPUT";
+        default: return "MLA_ERR_UNKNOWN";
+    }
+}
+
+size_t mla_metadata_ints(int num_sms) {
+    return num_sms < 1 ? 0 : (size_t)kMetaInts * ((size_t)num_sms + 1);
+}
+
+size_t mla_num_splits_len(int batch, int h_q, int s_q) {
+    if (!shape_ok(batch, h_q, s_q)) return 0;
+    return (size_t)batch * num_tiles(h_q, s_q) + 1;
+}
+
+size_t mla_workspace_bytes(int batch, int h_q, int s_q, int num_sms) {
+    if (!shape_ok(batch, h_q, s_q) || num_sms < 1) return 0;
+    const size_t cap = max_chunks_for(batch, h_q, s_q, num_sms);
+    return ws_o_offset(cap) + cap * kTileRows * kHeadDimV * 4 + kAlign;
+}
+
+int mla_num_work_units(int num_sms) {
+    if (num_sms < 1) return MLA_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    const int pairs = device_pairs(dev);
+    if (pairs < 1) return MLA_ERR_CUDA;
+    int u = num_sms / 2;
+    if (u > pairs) u = pairs;
+    return u < 1 ? 1 : u;
+}
+
+mla_status mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q, int num_sms,
+                            int32_t* metadata, int32_t* num_splits, void* stream) {
+    if (!seqlens || !metadata || !num_splits || num_sms < 1) return MLA_ERR_INVALID_ARG;
+    if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
+    const int units = mla_num_work_units(num_sms);
+    if (units < 0) return units;
+    metadata_kernel<<<1, kMetaThreads, 0, (cudaStream_t)stream>>>(
+        seqlens, batch, h_q, s_q, num_tiles(h_q, s_q), units, metadata, num_splits);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status mla_decode_fwd_simt(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                               const int32_t* block_table, int max_blocks,
+                               const int32_t* seqlens, int batch, int s_q, int h_q,
+                               float scale, int causal, const int32_t* metadata,
+                               const int32_t* num_splits, void* workspace,
+                               size_t workspace_bytes, uint16_t* out, float* lse,
+                               void* stream) {
+    mla_status st = validate_decode(q, kcache, num_blocks, block_table, max_blocks, seqlens,
+                                    batch, s_q, h_q, scale, causal, metadata, num_splits,
+                                    workspace, workspace_bytes, out, lse);
+    if (st != MLA_OK) return st;
+    DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
+                                 batch, s_q, h_q, scale, causal, metadata, num_splits,
+                                 workspace, workspace_bytes, out, lse);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    const int pairs = device_pairs(dev);
+    if (pairs < 1) return MLA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    decode_simt_kernel<<<2 * pairs, kSimtThreads, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    return launch_combine(p, s);
+}
+
+mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                          const int32_t* block_table, int max_blocks, const int32_t* seqlens,
+                          int batch, int s_q, int h_q, float scale, int causal,
+                          const int32_t* metadata, const int32_t* num_splits, void* workspace,
+                          size_t workspace_bytes, uint16_t* out, float* lse, void* stream) {
+    return mla_decode_fwd_simt(q, kcache, num_blocks, block_table, max_blocks, seqlens, batch,
+                               s_q, h_q, scale, causal, metadata, num_splits, workspace,
+                               workspace_bytes, out, lse, stream);
+}
+
+mla_status mla_get_last_device_error(void* stream, uint32_t* detail) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
+    uint32_t w = 0;
+    if (cudaMemcpyFromSymbol(&w, g_mla_error, sizeof(w)) != cudaSuccess) return MLA_ERR_CUDA;
+    if (detail) *detail = w;
+    if (w == 0) return MLA_OK;
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_mla_error, &zero, sizeof(zero)) != cudaSuccess) return MLA_ERR_CUDA;
+    return (w & 0xffu) == kErrTimeout ? MLA_ERR_DEVICE_TIMEOUT : MLA_ERR_DEVICE_BAD_INPUT;
+}
+
+mla_status mla_plan_host(const int32_t* seqlens_host, int batch, int h_q, int s_q,
+                         int num_units, int32_t* metadata_host, int32_t* num_splits_host) {
+    if (!seqlens_host || !metadata_host || !num_splits_host || num_units < 1)
+        return MLA_ERR_INVALID_ARG;
+    if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
+    const int tiles = num_tiles(h_q, s_q);
+    const int V = batch * tiles;
+    std::vector<int> nblk(V);
+    std::vector<int64_t> C(V + 1, 0);
+    for (int v = 0; v < V; ++v) {
+        const int L = seqlens_host[v % batch];
+        nblk[v] = pages_of(L < 0 ? 0 : L);
+        C[v + 1] = C[v] + kOverheadPages + nblk[v];
+    }
+    if (C[V] > 0x7fffffffLL) return MLA_ERR_UNSUPPORTED;
+    const int64_t W = unit_cost(C[V], num_units);
+    auto cost = [&](int v) { return C[v]; };
+    auto pages = [&](int v) { return nblk[v]; };
+    for (int u = 0; u < num_units; ++u) {
+        int vb, kb, ve, ke;
+        locate((int64_t)u * W, cost, pages, V, kOverheadPages, &vb, &kb);
+        locate((int64_t)(u + 1) * W, cost, pages, V, kOverheadPages, &ve, &ke);
+        int chunk = 0;
+        if (vb < V && (vb != ve || kb != ke)) chunk = u - unit_of(C[vb] + kOverheadPages, W);
+        int32_t* m = metadata_host + kMetaInts * (u + 1);
+        m[0] = vb; m[1] = kb; m[2] = ve; m[3] = ke; m[4] = chunk;
+        m[5] = 0; m[6] = 0; m[7] = 0;
+    }
+    metadata_host[0] = num_units; metadata_host[1] = tiles; metadata_host[2] = batch;
+    metadata_host[3] = h_q; metadata_host[4] = s_q; metadata_host[5] = (int32_t)W;
+    metadata_host[6] = 0; metadata_host[7] = 0;
+    int32_t acc = 0;
+    for (int v = 0; v < V; ++v) {
+        num_splits_host[v] = acc;
+        acc += chunks_of(C[v], nblk[v], W, kOverheadPages);
+    }
+    num_splits_host[V] = acc;
+    return MLA_OK;
+}
+
+}  // extern "C"

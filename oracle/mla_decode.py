@@ -73,14 +73,21 @@ def visible_tokens(seqlen: int, s_q: int, i: int, causal: bool) -> int:
     return seqlen - s_q + i + 1 if causal else seqlen
 
 
-def gather_tokens(kcache: np.ndarray, block_table_row: np.ndarray, n: int) -> np.ndarray:
-    """Dense [n, 576] copy of a sequence's first n cache rows through its block table.
+def gather_tokens(kcache, block_table_row, n: int) -> np.ndarray:
+    """Dense fp64 [n, 576] copy of a sequence's first n cache rows through its block table.
 
     Logical token t lives in physical block block_table_row[t // 64], slot t % 64
-    (paged kvcache with block size 64, FlashMLA release article).
+    (paged kvcache with block size 64, FlashMLA release article). `kcache` may be a
+    numpy array or a torch tensor of any float dtype; only the gathered rows are upcast.
     """
     t = np.arange(n)
-    return kcache[block_table_row[t // BLOCK_SIZE], t % BLOCK_SIZE, 0, :]
+    blocks = _i64(block_table_row)[t // BLOCK_SIZE]
+    slots = t % BLOCK_SIZE
+    if hasattr(kcache, "detach"):
+        import torch
+        rows = kcache[torch.from_numpy(blocks), torch.from_numpy(slots), 0, :]
+        return _f64(rows)
+    return np.asarray(kcache, dtype=np.float64)[blocks, slots, 0, :]
 
 
 def decode(q, kcache, block_table, seqlens, scale: float, causal: bool,
@@ -91,12 +98,11 @@ def decode(q, kcache, block_table, seqlens, scale: float, causal: bool,
     seqlens [b]. Returns (out [b', s_q, h_q, 512], lse [b', h_q, s_q]) as float64,
     where b' runs over `batch_indices` (all sequences by default).
     """
-    kc = _f64(kcache)
     bt = _i64(block_table)
     lens = _i64(seqlens)
-    qq = _f64(q)
-    _, s_q, h_q, _ = qq.shape
-    idx = range(qq.shape[0]) if batch_indices is None else list(batch_indices)
+    _, s_q, h_q, _ = q.shape
+    idx = range(q.shape[0]) if batch_indices is None else list(batch_indices)
+    qq = _f64(q[list(idx)] if hasattr(q, "detach") else np.asarray(q)[list(idx)])
     out = np.zeros((len(idx), s_q, h_q, HEAD_DIM_V))
     lse = np.full((len(idx), h_q, s_q), -np.inf)
     for ob, b in enumerate(idx):
@@ -104,13 +110,13 @@ def decode(q, kcache, block_table, seqlens, scale: float, causal: bool,
         n_max = max(visible_tokens(L, s_q, i, causal) for i in range(s_q))
         if n_max <= 0:
             continue
-        K = gather_tokens(kc, bt[b], n_max)          # [n_max, 576]
+        K = gather_tokens(kcache, bt[b], n_max)      # [n_max, 576]
         V = K[:, :HEAD_DIM_V]                         # V = first 512 dims of the row
         for i in range(s_q):
             n = visible_tokens(L, s_q, i, causal)
             if n <= 0:
                 continue
-            S = scale * (qq[b, i] @ K[:n].T)          # [h_q, n]
+            S = scale * (qq[ob, i] @ K[:n].T)         # [h_q, n]
             m = S.max(axis=1, keepdims=True)
             E = np.exp(S - m)
             l = E.sum(axis=1)

@@ -1,0 +1,223 @@
+"""GPU parity of the CUDA decode path against the fp64 CPU oracle, through the C ABI.
+
+Tolerances (the decode's accuracy contract): max |out - oracle| <= 1e-2 on the bf16
+output and max |lse - oracle| <= 1e-3 on the fp32 log-sum-exp. Small cases compare every
+element; the full-size workloads run in the benchmark's launch configuration (all SMs)
+and compare sampled sequences the oracle computes one by one, plus properties that hold
+at any size (finite outputs, agreement with the no-split schedule).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_paged_kv_06_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+ATOL_OUT = 1e-2
+ATOL_LSE = 1e-3
+
+
+def _mla():
+    from mla_paged_kv_06_b200 import mla
+    return mla
+
+
+def to_dev(x):
+    return dict(q=x.q.cuda(), kcache=x.kcache.cuda(), block_table=x.block_table.cuda(),
+                seqlens=x.seqlens.cuda())
+
+
+def run(x, d=None, impl="tc", num_sms=None, check_error=True):
+    mla = _mla()
+    d = d or to_dev(x)
+    nsm = num_sms or mla.default_num_sms()
+    meta, ns = mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm)
+    fn = mla.mla_decode_fwd if impl == "tc" else mla.mla_decode_fwd_simt
+    out, lse = fn(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale, x.causal,
+                  meta, ns, num_sms=nsm)
+    torch.cuda.synchronize()
+    if check_error:
+        st, word = mla.mla_get_last_device_error()
+        assert st == 0, f"device error {mla.status_string(st)} word={word:#x}"
+    return out, lse
+
+
+def compare(out, lse, ref_out, ref_lse, what=""):
+    o = out.double().cpu().numpy()
+    l = lse.double().cpu().numpy()
+    assert np.isfinite(o).all(), f"{what}: non-finite output"
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(np.isneginf(l), ~fin), f"{what}: empty-row lse mismatch"
+    d_o = np.abs(o - ref_out).max() if o.size else 0.0
+    d_l = np.abs(l[fin] - ref_lse[fin]).max() if fin.any() else 0.0
+    assert d_o <= ATOL_OUT, f"{what}: max|dout|={d_o:.3e}"
+    assert d_l <= ATOL_LSE, f"{what}: max|dlse|={d_l:.3e}"
+    return d_o, d_l
+
+
+def oracle_all(x):
+    return oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale, x.causal)
+
+
+@pytest.mark.parametrize("impl", ["tc", "simt"])
+def test_tiny_workload_parity(impl):
+    x = wl.make_workload("tiny")
+    out, lse = run(x, impl=impl)
+    assert tuple(out.shape) == (2, 1, 16, 512) and tuple(lse.shape) == (2, 16, 1)
+    compare(out, lse, *oracle_all(x), what=f"tiny/{impl}")
+
+
+SMALL = [
+    # lens, s_q, h_q, causal
+    ([1, 63, 64, 65, 127, 128, 129], 1, 16, False),
+    ([700, 1, 2000, 64], 1, 128, False),
+    ([513, 4096, 1000], 2, 128, True),
+    ([300, 65, 2], 2, 64, True),
+    ([1500, 333], 1, 64, False),
+    ([17, 200, 190], 4, 32, True),
+    ([129, 5], 1, 1, False),
+    ([258, 3, 1, 0, 64], 3, 7, True),
+    ([2500], 1, 100, False),
+]
+
+
+@pytest.mark.parametrize("case", SMALL)
+@pytest.mark.parametrize("num_sms", [None, 1, 6])
+@pytest.mark.parametrize("impl", ["tc", "simt"])
+def test_small_parity(case, num_sms, impl):
+    lens, s_q, h_q, causal = case
+    x = wl.make_paged_inputs(lens, s_q, h_q, seed=sum(lens) + s_q, causal=causal,
+                             spare_blocks=3, poison=True)
+    out, lse = run(x, impl=impl, num_sms=num_sms)
+    compare(out, lse, *oracle_all(x), what=f"{case}/{num_sms}/{impl}")
+
+
+def test_device_metadata_matches_host_plan():
+    mla = _mla()
+    for lens, h_q, s_q in [([37, 130], 16, 1), ([65536, 10, 0, 65536, 3], 64, 1),
+                           ([8192] * 128, 128, 2), (list(range(0, 9000, 37)), 128, 1)]:
+        seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        for nsm in [1, 2, 13, mla.default_num_sms()]:
+            meta, ns = mla.mla_get_metadata(seq, h_q, s_q, nsm)
+            units = mla.mla_num_work_units(nsm)
+            hm, hns = mla.mla_plan_host(lens, h_q, s_q, units)
+            assert np.array_equal(meta.cpu().numpy()[: hm.size], hm)
+            assert np.array_equal(ns.cpu().numpy(), hns)
+
+
+FULL = ["uniform", "v3", "spec", "skewed"]
+
+
+def _sample(x, k=6):
+    lens = x.seqlens.tolist()
+    order = sorted(range(len(lens)), key=lambda b: lens[b])
+    g = np.random.default_rng(7)
+    pick = {order[0], order[-1], order[len(order) // 2]}
+    pick |= set(g.choice(len(lens), size=min(k, len(lens)), replace=False).tolist())
+    return sorted(pick)
+
+
+@pytest.fixture(scope="module")
+def full_inputs():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            cache.clear()
+            x = wl.make_workload(name, seed=0)
+            cache[name] = (x, to_dev(x))
+        return cache[name]
+    return get
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload_sampled_parity(name, full_inputs):
+    x, d = full_inputs(name)
+    out, lse = run(x, d)
+    o = out.double().cpu().numpy()
+    assert np.isfinite(o).all()
+    idx = _sample(x)
+    ref_out, ref_lse = oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale,
+                                     x.causal, batch_indices=idx)
+    compare(out[idx], lse[idx], ref_out, ref_lse, what=name)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload_split_matches_no_split(name, full_inputs):
+    x, d = full_inputs(name)
+    out_a, lse_a = run(x, d)
+    out_b, lse_b = run(x, d, num_sms=1)
+    assert (out_a.float() - out_b.float()).abs().max().item() <= ATOL_OUT
+    assert (lse_a - lse_b).abs().max().item() <= ATOL_LSE
+
+
+def test_full_workload_tc_matches_simt(full_inputs):
+    x, d = full_inputs("skewed")
+    out_a, lse_a = run(x, d, impl="tc")
+    out_b, lse_b = run(x, d, impl="simt")
+    assert (out_a.float() - out_b.float()).abs().max().item() <= ATOL_OUT
+    assert (lse_a - lse_b).abs().max().item() <= ATOL_LSE
+
+
+def test_nan_poison_full_size():
+    x = wl.make_workload("v3", seed=3, poison=True)
+    assert torch.isnan(x.kcache[:, :, 0, 0].float()).any()
+    out, lse = run(x)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    idx = _sample(x, 3)
+    ref = oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale, x.causal,
+                        batch_indices=idx)
+    compare(out[idx], lse[idx], *ref, what="v3-poison")
+
+
+@pytest.mark.parametrize("impl", ["tc", "simt"])
+def test_block_permutation_is_bit_exact(impl):
+    x = wl.make_paged_inputs([130, 4000, 64, 1], 2, 128, seed=5, causal=True,
+                             spare_blocks=2, poison=True)
+    out, lse = run(x, impl=impl)
+    g = torch.Generator().manual_seed(4)
+    perm = torch.randperm(x.num_blocks, generator=g)
+    kc2 = torch.empty_like(x.kcache)
+    kc2[perm] = x.kcache
+    bt2 = perm[x.block_table.long()].to(torch.int32)
+    y = wl.DecodeInputs(x.q, kc2, bt2, x.seqlens, x.scale, x.causal, "perm", 5)
+    out2, lse2 = run(y, impl=impl)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def test_repeat_runs_are_bit_identical():
+    x = wl.make_paged_inputs([3000, 17, 900], 1, 128, seed=8)
+    d = to_dev(x)
+    a = run(x, d)
+    b = run(x, d)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_single_token_returns_v_row_exactly():
+    x = wl.make_paged_inputs([1, 1, 1], 1, 128, seed=9)
+    out, lse = run(x)
+    for b in range(3):
+        row = x.kcache[int(x.block_table[b, 0]), 0, 0, :512]
+        assert torch.equal(out[b, 0].cpu(), row.expand(128, 512))
+
+
+def test_bad_inputs_report_device_error():
+    mla = _mla()
+    x = wl.make_paged_inputs([100, 50], 1, 16, seed=10)
+    d = to_dev(x)
+    # a block id past the pool: recorded, skipped, no fault
+    d["block_table"][0, 1] = x.num_blocks + 5
+    run(x, d, check_error=False)
+    st, word = mla.mla_get_last_device_error()
+    assert st == mla.MLA_ERR_DEVICE_BAD_INPUT, (st, hex(word))
+    # a length the block table cannot hold: recorded and clamped
+    d = to_dev(x)
+    d["seqlens"][1] = 64 * x.block_table.shape[1] + 1
+    run(x, d, check_error=False)
+    st, _ = mla.mla_get_last_device_error()
+    assert st == mla.MLA_ERR_DEVICE_BAD_INPUT
+    st, _ = mla.mla_get_last_device_error()
+    assert st == mla.MLA_OK
