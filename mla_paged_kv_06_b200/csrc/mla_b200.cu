@@ -1,5 +1,6 @@
 // libmla_b200.so: the C ABI of include/mla.h. This is the library's single translation
 // unit; the kernels live in the headers it includes.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -13,6 +14,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "decode_simt.cuh"
+#include "decode_sm100.cuh"
 #include "metadata.cuh"
 #include "sched.cuh"
 
@@ -46,18 +48,90 @@ size_t ws_capacity(size_t bytes) {
 
 size_t ws_o_offset(size_t cap) { return align_up(kWsHeader + cap * kTileRows * 4, kAlign); }
 
-// SM pairs the decode can keep co-resident on a device (cached per device).
+// Opt the split kernel into its shared-memory footprint (once per device).
+bool prepare_sm100_kernel(int dev) {
+    static std::mutex mu;
+    static std::vector<char> done;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)done.size() <= dev) done.resize(dev + 1, 0);
+    if (done[dev]) return true;
+    if (cudaFuncSetAttribute(sm100::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm100::kSmemAlloc) != cudaSuccess)
+        return false;
+    done[dev] = 1;
+    return true;
+}
+
+// 2-CTA clusters of the split kernel that can be co-resident on a device (cached per
+// device); a schedule never uses more units than this, so every unit runs in one wave.
 int device_pairs(int dev) {
     static std::mutex mu;
     static std::vector<int> cache;
-    std::lock_guard<std::mutex> lock(mu);
-    if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
-    if (cache[dev] > 0) return cache[dev];
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if ((int)cache.size() > dev && cache[dev] > 0) return cache[dev];
+    }
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return -1;
-    cache[dev] = sms / 2 < 1 ? 1 : sms / 2;
-    return cache[dev];
+    int pairs = sms / 2 < 1 ? 1 : sms / 2;
+    if (prepare_sm100_kernel(dev)) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * pairs);
+        cfg.blockDim = dim3(sm100::kThreads);
+        cfg.dynamicSmemBytes = sm100::kSmemAlloc;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, sm100::decode_kernel, &cfg) == cudaSuccess &&
+            clusters > 0 && clusters < pairs)
+            pairs = clusters;
+        cudaGetLastError();
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+    cache[dev] = pairs;
+    return pairs;
+}
+
+// cuTensorMapEncodeTiled from the driver, found at run time so the library does not
+// link libcuda (it must load on machines without a GPU driver).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2D view of the page pool: [num_blocks * 64 rows][576 bf16], row stride 1152 bytes.
+bool make_pool_map(CUtensorMap* map, const void* kcache, int num_blocks, int box_cols,
+                   CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)num_blocks * kBlock};
+    const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)kBlock};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kcache), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 mla_status validate_decode(const uint16_t* q, const uint16_t* kcache, int num_blocks,
@@ -200,9 +274,25 @@ mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blo
                           int batch, int s_q, int h_q, float scale, int causal,
                           const int32_t* metadata, const int32_t* num_splits, void* workspace,
                           size_t workspace_bytes, uint16_t* out, float* lse, void* stream) {
-    return mla_decode_fwd_simt(q, kcache, num_blocks, block_table, max_blocks, seqlens, batch,
-                               s_q, h_q, scale, causal, metadata, num_splits, workspace,
-                               workspace_bytes, out, lse, stream);
+    mla_status st = validate_decode(q, kcache, num_blocks, block_table, max_blocks, seqlens,
+                                    batch, s_q, h_q, scale, causal, metadata, num_splits,
+                                    workspace, workspace_bytes, out, lse);
+    if (st != MLA_OK) return st;
+    DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
+                                 batch, s_q, h_q, scale, causal, metadata, num_splits,
+                                 workspace, workspace_bytes, out, lse);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    const int pairs = device_pairs(dev);
+    if (pairs < 1 || !prepare_sm100_kernel(dev)) return MLA_ERR_CUDA;
+    CUtensorMap tm_lat, tm_rope;
+    if (!make_pool_map(&tm_lat, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_pool_map(&tm_rope, kcache, num_blocks, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+        return MLA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    sm100::decode_kernel<<<2 * pairs, sm100::kThreads, sm100::kSmemAlloc, s>>>(p, tm_lat, tm_rope);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    return launch_combine(p, s);
 }
 
 mla_status mla_get_last_device_error(void* stream, uint32_t* detail) {
