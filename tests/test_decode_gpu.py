@@ -18,6 +18,10 @@ pytestmark = pytest.mark.gpu
 
 ATOL_OUT = 1e-2
 ATOL_LSE = 1e-3
+# Two GPU results that are each within the tolerance of the oracle can differ by twice
+# it (one bf16 ulp is 0.0156 at |o| in [2, 4)), so GPU-vs-GPU comparisons use 2x.
+ATOL_PAIR_OUT = 2 * ATOL_OUT
+ATOL_PAIR_LSE = 2 * ATOL_LSE
 
 
 def _mla():
@@ -150,16 +154,16 @@ def test_full_workload_split_matches_no_split(name, full_inputs):
     x, d = full_inputs(name)
     out_a, lse_a = run(x, d)
     out_b, lse_b = run(x, d, num_sms=1)
-    assert (out_a.float() - out_b.float()).abs().max().item() <= ATOL_OUT
-    assert (lse_a - lse_b).abs().max().item() <= ATOL_LSE
+    assert (out_a.float() - out_b.float()).abs().max().item() <= ATOL_PAIR_OUT
+    assert (lse_a - lse_b).abs().max().item() <= ATOL_PAIR_LSE
 
 
 def test_full_workload_tc_matches_simt(full_inputs):
     x, d = full_inputs("skewed")
     out_a, lse_a = run(x, d, impl="tc")
     out_b, lse_b = run(x, d, impl="simt")
-    assert (out_a.float() - out_b.float()).abs().max().item() <= ATOL_OUT
-    assert (lse_a - lse_b).abs().max().item() <= ATOL_LSE
+    assert (out_a.float() - out_b.float()).abs().max().item() <= ATOL_PAIR_OUT
+    assert (lse_a - lse_b).abs().max().item() <= ATOL_PAIR_LSE
 
 
 def test_nan_poison_full_size():
