@@ -7,19 +7,30 @@
 // the pair splits the 576 dims: CTA c holds latent dims [256c, 256c+256) and rope dims
 // [512+32c, 512+32c+32) of q and of every page, computes the partial scores over its
 // 288 dims, and owns output columns [256c, 256c+256). The two partial score tiles are
-// exchanged over distributed shared memory and summed identically in both CTAs, so
-// both run the same online softmax and no FLOP or HBM byte is duplicated.
+// exchanged through distributed shared memory, so no FLOP or HBM byte is duplicated.
+// Shared-memory traffic between SMs is slow (about 15 B/clock/SM for bulk copies), so
+// each row's 64 partial scores travel as 16-bit fixed point with a per-row scale (the
+// row's largest magnitude over its visible tokens maps to 32767): 16.5 KB per page
+// instead of 32 KB, error at most 2^-16 of that magnitude. Each CTA adds the peer's
+// dequantised partial to its own exact fp32 partial.
 //
-// Per CTA (192 threads):
-//   warp 0   TMA producer: page ids from the block table, 4 SW128 latent boxes + 1 SW64
-//            rope box per page into a 4-stage ring.
-//   warp 1   TMEM owner and MMA issuer (one thread): S = Q K^T (M=128, N=64, K=288;
-//            the latent part reads Q from TMEM, the rope part from shared memory) and
-//            O += P V (M=128, N=256, K=64; P from TMEM, V = the page's latent boxes
-//            read MN-major), completion tracked with tcgen05.commit.
-//   warps 2-5 softmax / correction / epilogue, one thread per query row.
-// TMEM columns: O [0,256) fp32, Q latent [256,384) bf16x2, S0 [384,448), S1 [448,512);
-// P (bf16x2) overwrites the first 32 columns of the S buffer it came from.
+// Per CTA (384 threads, three warpgroups whose registers are rebalanced at start):
+//   warps 0-3 softmax / correction / epilogue, one thread per query row (TMEM lane).
+//             While page j is combined and exponentiated, page j+1's scores are already
+//             read (and, by the senders, on their way to the peer).
+//   warps 4-7 senders: read each page's partial scores from TMEM, quantise them into a
+//             local staging buffer and bulk-copy it into the peer's exchange buffer;
+//             relay to the peer when this CTA's softmax has finished reading an exchange
+//             buffer. Remote traffic never stalls the softmax warps.
+//   warp 8    TMA producer: page ids from the block table, 4 SW128 latent boxes + 1 SW64
+//             rope box per page into a 4-stage ring.
+//   warp 9    TMEM owner and MMA issuer (one thread): S = Q K^T (M=128, N=64, K=288;
+//             the latent part reads Q from TMEM, the rope part from shared memory) and
+//             O += P V (M=128, N=256, K=64; P from TMEM, V = the page's latent boxes
+//             read MN-major). QK runs two pages ahead of PV.
+//   warps 10-11 idle (they complete the third warpgroup).
+// TMEM columns: O [0,256) fp32, Q latent [256,384) bf16x2, S [384,448) fp32,
+// P0 [448,480) and P1 [480,512) bf16x2. S is released as soon as both groups read it.
 // Scores stay in the log2 domain (scale * log2 e folded in). The running max is only
 // raised when a new score exceeds it by more than kRescaleLog2, so O is rescaled rarely.
 #pragma once
@@ -30,7 +41,15 @@
 namespace mla {
 namespace sm100 {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
+constexpr int kWarpSender0 = 4;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+// Registers per thread after rebalancing: 128 * (240 + 104 + 56) = 51200, within the
+// 384 * 168 = 64512 the CTA is launched with (ptxas reports 168 for this kernel).
+constexpr uint32_t kRegsSoftmax = 240;
+constexpr uint32_t kRegsSender = 104;
+constexpr uint32_t kRegsControl = 56;
 constexpr int kStages = 4;
 constexpr int kLatentHalf = 256;                     // latent dims per CTA
 constexpr int kRopeHalf = 32;                        // rope dims per CTA
@@ -38,24 +57,33 @@ constexpr uint32_t kBoxBytes = 64 * 64 * 2;          // one SW128 box: 64 tokens
 constexpr uint32_t kRopeBoxBytes = 64 * 32 * 2;      // one SW64 box: 64 tokens x 32 dims
 constexpr uint32_t kStageBytes = 4 * kBoxBytes + kRopeBoxBytes;   // 36 KB
 constexpr uint32_t kQropeBytes = 128 * kRopeHalf * 2;             // 8 KB
-constexpr uint32_t kXRowStride = 272;                // 64 fp32 + 16 B pad: no bank conflicts
-constexpr uint32_t kXBytes = 128 * kXRowStride;
+// Exchange buffer (and its staging twin): 128 rows x 64 biased 16-bit scores (128 B per
+// row, 16-byte chunks XOR-swizzled by row % 8 so row-per-thread access is conflict-free)
+// followed by the 128 per-row fp32 scales.
+constexpr uint32_t kXDataBytes = 128 * 128;
+constexpr uint32_t kXBytes = kXDataBytes + 128 * 4;  // 16896
+constexpr uint32_t kXPayload = kXBytes;              // bytes the peer sends per page
+constexpr float kQuantMax = 32767.f;
 
 constexpr uint32_t kOffStage = 0;
 constexpr uint32_t kOffQrope = kStages * kStageBytes;
-constexpr uint32_t kOffX = kOffQrope + kQropeBytes;
-constexpr uint32_t kOffBar = kOffX + 2 * kXBytes;
+constexpr uint32_t kOffX = kOffQrope + kQropeBytes;          // [2] receive buffers
+constexpr uint32_t kOffXStage = kOffX + 2 * kXBytes;         // [2] staging buffers
+constexpr uint32_t kOffBar = kOffXStage + 2 * kXBytes;
 // barriers (8 B each)
 enum : uint32_t {
     kBarFull = 0,                     // [kStages] TMA -> MMA
     kBarEmpty = kBarFull + kStages,   // [kStages] MMA (PV done) -> TMA
-    kBarSFull = kBarEmpty + kStages,  // [2] QK done -> softmax
-    kBarPReady = kBarSFull + 2,       // [2] P written -> MMA
-    kBarPvDone = kBarPReady + 2,      // [2] PV done -> MMA / softmax
-    kBarXFull = kBarPvDone + 2,       // [2] peer scores arrived
-    kBarXFree = kBarXFull + 2,        // [2] peer finished reading what we sent
+    kBarSFull = kBarEmpty + kStages,  // QK done -> softmax and senders
+    kBarSFree = kBarSFull + 1,        // softmax and senders read S -> MMA
+    kBarPReady = kBarSFree + 1,       // [2] P written -> MMA
+    kBarPvDone = kBarPReady + 2,      // [2] PV done -> softmax
+    kBarXFull = kBarPvDone + 2,       // [2] peer scores landed (tx count)
+    kBarXRead = kBarXFull + 2,        // [2] softmax read exchange buffer -> senders
+    kBarXFree = kBarXRead + 2,        // [2] peer's softmax read what we sent
     kBarQReady = kBarXFree + 2,       // query tile in TMEM / smem
-    kNumBars = kBarQReady + 1
+    kBarStage = kBarQReady + 1,       // [2] staging buffer written -> sending thread
+    kNumBars = kBarStage + 2
 };
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16;
@@ -64,7 +92,8 @@ constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;      // room to align the bas
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;
 constexpr uint32_t kColQ = 256;
-constexpr uint32_t kColS = 384;                          // + 64 * buffer
+constexpr uint32_t kColS = 384;
+constexpr uint32_t kColP = 448;                          // + 32 * buffer
 
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -106,9 +135,9 @@ __device__ __forceinline__ bool wait_bar(const Shared& sh, uint32_t bar, uint32_
     }
 }
 
-// Warp-uniform bounded wait for the softmax warps: every lane waits, and the warp
-// proceeds only if all lanes saw the phase complete, so no lane can leave a loop whose
-// body holds .sync.aligned tcgen05 instructions while its neighbours stay in it.
+// Warp-uniform bounded wait: every lane waits, and the warp proceeds only if all lanes
+// saw the phase complete, so no lane can leave a loop whose body holds .sync.aligned
+// tcgen05 instructions while its neighbours stay in it.
 template <bool kCluster>
 __device__ __forceinline__ bool warp_wait_bar(const Shared& sh, uint32_t bar, uint32_t parity,
                                               uint32_t where) {
@@ -161,7 +190,7 @@ struct ItemIter {
     }
 };
 
-// ------------------------------------------------------------------ producer (warp 0)
+// ------------------------------------------------------------------ producer (warp 8)
 __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared& sh,
                                              const CUtensorMap* tm_lat, const CUtensorMap* tm_rope,
                                              uint32_t crank) {
@@ -187,7 +216,8 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             const uint32_t dst = sh.stage(s);
             const int y = pid * kBlock;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) ptx::tma_load_2d(dst + i * kBoxBytes, tm_lat, full, x_lat + 64 * i, y);
+            for (int i = 0; i < 4; ++i)
+                ptx::tma_load_2d(dst + i * kBoxBytes, tm_lat, full, x_lat + 64 * i, y);
             ptx::tma_load_2d(dst + 4 * kBoxBytes, tm_rope, full, x_rope, y);
         }
     }
@@ -198,84 +228,303 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
     }
 }
 
-// ------------------------------------------------------------------ MMA issuer (warp 1)
+// ------------------------------------------------------------------ MMA issuer (warp 9)
+// S = Q K^T for global page index G (stage G % kStages).
+__device__ __forceinline__ bool issue_qk(const Shared& sh, uint32_t tmem, uint32_t G) {
+    const uint32_t s = G % kStages;
+    if (!wait_bar<false>(sh, sh.bar(kBarFull + s), (G / kStages) & 1u, 0x21u)) return false;
+    if (G >= 1 && !wait_bar<false>(sh, sh.bar(kBarSFree), (G - 1) & 1u, 0x22u)) return false;
+    ptx::tc_fence_after();
+    const uint32_t d = tmem + kColS;
+    const uint32_t st = sh.stage(s);
+    const uint32_t qrope = sh.base_u32 + kOffQrope;
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+        const uint64_t bdesc =
+            ptx::smem_desc(st + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024, 2);
+        ptx::mma_ts(d, tmem + kColQ + 8 * kk, bdesc, kIdescQK, kk > 0);
+    }
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+        const uint64_t adesc = ptx::smem_desc(qrope + 32 * kk, 16, 512, 4);
+        const uint64_t bdesc = ptx::smem_desc(st + 4 * kBoxBytes + 32 * kk, 16, 512, 4);
+        ptx::mma_ss(d, adesc, bdesc, kIdescQK, 1);
+    }
+    ptx::mma_commit(sh.bar(kBarSFull));
+    return true;
+}
+
+// O += P V for global page index G; `first` starts a new accumulation.
+__device__ __forceinline__ bool issue_pv(const Shared& sh, uint32_t tmem, uint32_t G, bool first) {
+    const uint32_t pb = G & 1u;
+    if (!wait_bar<false>(sh, sh.bar(kBarPReady + pb), (G >> 1) & 1u, 0x23u)) return false;
+    ptx::tc_fence_after();
+    const uint32_t st = sh.stage(G % kStages);
+    const uint32_t a = tmem + kColP + 32 * pb;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bdesc = ptx::smem_desc(st + kk * 2048, kBoxBytes, 1024, 2);
+        ptx::mma_ts(tmem + kColO, a + 8 * kk, bdesc, kIdescPV, (!first || kk > 0) ? 1u : 0u);
+    }
+    ptx::mma_commit(sh.bar(kBarPvDone + pb));
+    ptx::mma_commit(sh.bar(kBarEmpty + G % kStages));
+    return true;
+}
+
 __device__ __forceinline__ void run_mma(const DecodeParams& p, const Shared& sh, uint32_t tmem) {
     ItemIter iter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item it;
-    uint32_t g = 0;        // pages consumed (stage ring position)
-    uint32_t G = 0;        // blocks processed (S/P buffer position), same as g here
+    uint32_t G = 0;        // global page index (stage ring and S/P buffers)
     uint32_t items = 0;
-    const uint32_t qrope = sh.base_u32 + kOffQrope;
     while (iter.next(it)) {
         if (!wait_bar<false>(sh, sh.bar(kBarQReady), items & 1u, 0x20u)) return;
         ptx::tc_fence_after();
-        const int n = it.k_hi - it.k_lo;
-        for (int j = 0; j <= n; ++j) {
-            if (j < n) {
-                // S[G % 2] = Q K^T over this CTA's 288 dims
-                const uint32_t s = g % kStages;
-                const uint32_t sb = G & 1u;
-                if (!wait_bar<false>(sh, sh.bar(kBarFull + s), (g / kStages) & 1u, 0x21u)) return;
-                if (G >= 2 && !wait_bar<false>(sh, sh.bar(kBarPvDone + sb), ((G - 2) >> 1) & 1u, 0x22u))
-                    return;
-                ptx::tc_fence_after();
-                const uint32_t d = tmem + kColS + 64 * sb;
-                const uint32_t st = sh.stage(s);
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const uint64_t bdesc = ptx::smem_desc(st + (kk >> 2) * kBoxBytes + (kk & 3) * 32,
-                                                          16, 1024, 2);
-                    ptx::mma_ts(d, tmem + kColQ + 8 * kk, bdesc, kIdescQK, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                    const uint64_t adesc = ptx::smem_desc(qrope + 32 * kk, 16, 512, 4);
-                    const uint64_t bdesc = ptx::smem_desc(st + 4 * kBoxBytes + 32 * kk, 16, 512, 4);
-                    ptx::mma_ss(d, adesc, bdesc, kIdescQK, 1);
-                }
-                ptx::mma_commit(sh.bar(kBarSFull + sb));
-            }
-            if (j >= 1) {
-                // O += P V for the previous page
-                const uint32_t Gp = G - 1;
-                const uint32_t gp = g - 1;
-                const uint32_t sbp = Gp & 1u;
-                if (!wait_bar<false>(sh, sh.bar(kBarPReady + sbp), (Gp >> 1) & 1u, 0x23u)) return;
-                ptx::tc_fence_after();
-                const uint32_t st = sh.stage(gp % kStages);
-                const uint32_t a = tmem + kColS + 64 * sbp;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bdesc = ptx::smem_desc(st + kk * 2048, kBoxBytes, 1024, 2);
-                    ptx::mma_ts(tmem + kColO, a + 8 * kk, bdesc, kIdescPV, (j > 1 || kk > 0) ? 1u : 0u);
-                }
-                ptx::mma_commit(sh.bar(kBarPvDone + sbp));
-                ptx::mma_commit(sh.bar(kBarEmpty + gp % kStages));
-            }
-            if (j < n) { ++g; ++G; }
+        const uint32_t n = (uint32_t)(it.k_hi - it.k_lo);
+        // QK runs two pages ahead of PV: S of page j+1 is read (freeing the single S
+        // buffer) before P of page j exists, so QK(j+2) can be issued ahead of PV(j).
+        if (!issue_qk(sh, tmem, G)) return;
+        if (n > 1 && !issue_qk(sh, tmem, G + 1)) return;
+        for (uint32_t j = 0; j < n; ++j) {
+            if (j + 2 < n && !issue_qk(sh, tmem, G + j + 2)) return;
+            if (!issue_pv(sh, tmem, G + j, j == 0)) return;
         }
+        G += n;
         ++items;
     }
 }
 
-// ------------------------------------------------------------------ softmax (warps 2-5)
+// ------------------------------------------------------------------ senders (warps 4-7)
+// For every page G: read this CTA's partial scores (one TMEM lane per thread), release S,
+// quantise the row to 16-bit fixed point, write it into staging buffer G % 2 and (one
+// thread) bulk-copy the buffer into the peer's exchange buffer G % 2, completing tx bytes
+// on the peer's kBarXFull. Before reusing buffer G % 2, wait until the peer's softmax has
+// read what was sent into it two pages earlier (kBarXFree, arrived by the peer's
+// senders; the copy out of our staging buffer is then complete too), and forward this
+// CTA's own "buffer read" signal to the peer in the same way.
+__device__ __forceinline__ void run_sender(const DecodeParams& p, const Shared& sh, uint32_t tmem,
+                                           uint32_t crank, int quarter, int lane) {
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t peer = crank ^ 1u;
+    const uint32_t x_peer = ptx::mapa(sh.base_u32 + kOffX, peer);
+    const uint32_t xfull_peer = ptx::mapa(sh.bar(kBarXFull), peer);
+    const uint32_t xfree_peer = ptx::mapa(sh.bar(kBarXFree), peer);
+    const bool leader = row == 0;
+
+    ItemIter iter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
+    Item it;
+    uint32_t G = 0;
+    while (iter.next(it)) {
+        const int r = it.t * kTileRows + row;
+        const int n_vis = r < p.rows ? visible_tokens(it.L, p.s_q, r / p.h_q, p.causal) : 0;
+        const uint32_t n = (uint32_t)(it.k_hi - it.k_lo);
+        for (uint32_t j = 0; j < n; ++j, ++G) {
+            const uint32_t xb = G & 1u;
+            if (!warp_wait_bar<false>(sh, sh.bar(kBarSFull), G & 1u, 0x40u)) return;
+            ptx::tc_fence_after();
+            uint32_t sv[64];
+            ptx::tmem_ld64(tmem + lane_base + kColS, sv);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(sh.bar(kBarSFree));
+
+            // per-row scale over the visible tokens of this page
+            const int lim = n_vis - (it.k_lo + (int)j) * kBlock;
+            float mx = 0.f;
+            if (__all_sync(0xffffffffu, lim >= 64)) {
+#pragma unroll
+                for (int q = 0; q < 64; ++q) mx = fmaxf(mx, fabsf(__uint_as_float(sv[q])));
+            } else {
+#pragma unroll
+                for (int q = 0; q < 64; ++q)
+                    if (q < lim) mx = fmaxf(mx, fabsf(__uint_as_float(sv[q])));
+            }
+            const float inv = mx > 0.f ? kQuantMax / mx : 0.f;
+            // round to the nearest integer on the FMA pipe: adding 1.5 * 2^23 + 32768 leaves
+            // 32768 + round(x) (in [1, 65535] for |x| <= 32767) in the low 16 mantissa bits;
+            // masked columns may carry any code, the softmax never uses them
+            uint32_t pk[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const uint32_t ua = __float_as_uint(fmaf(__uint_as_float(sv[2 * q]), inv, 12615680.f));
+                const uint32_t ub = __float_as_uint(fmaf(__uint_as_float(sv[2 * q + 1]), inv, 12615680.f));
+                pk[q] = __byte_perm(ua, ub, 0x5410);
+            }
+
+            if (G >= 2) {
+                // relay: our softmax has read buffer xb (page G-2); the peer may refill it
+                if (leader) {
+                    if (!wait_bar<false>(sh, sh.bar(kBarXRead + xb), ((G - 2) >> 1) & 1u, 0x41u))
+                        return;
+                    ptx::mbar_arrive_remote(xfree_peer + 8 * xb);
+                }
+                // and the peer must have read our previous send into its buffer xb
+                if (!warp_wait_bar<true>(sh, sh.bar(kBarXFree + xb), ((G - 2) >> 1) & 1u, 0x42u))
+                    return;
+            }
+            const uint32_t stg = sh.base_u32 + kOffXStage + xb * kXBytes;
+            const uint32_t rowp = stg + (uint32_t)row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t phys = (uint32_t)(c ^ (row & 7));
+                ptx::st_shared_v4(rowp + phys * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                                  pk[4 * c + 3]);
+            }
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + kXDataBytes + 4 * row),
+                         "f"(mx * (1.f / kQuantMax)) : "memory");
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(sh.bar(kBarStage + xb));
+            if (leader) {
+                if (!wait_bar<false>(sh, sh.bar(kBarStage + xb), (G >> 1) & 1u, 0x43u)) return;
+                ptx::bulk_copy_to_peer(x_peer + xb * kXBytes, stg, kXBytes, xfull_peer + 8 * xb);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ softmax (warps 0-3)
 __device__ __forceinline__ float f32(uint32_t x) { return __uint_as_float(x); }
+
+struct RowState {
+    float m_ref;     // reference max (log2 domain); -inf until a visible token is seen
+    float l_sum;     // sum of 2^(s - m_ref) over the tokens seen
+};
+
+// Waits for S of page G, reads it into `sv` and releases the S buffer.
+__device__ __forceinline__ bool load_scores(const Shared& sh, uint32_t tmem, uint32_t lane_base,
+                                            uint32_t G, uint32_t* sv) {
+    if (!warp_wait_bar<false>(sh, sh.bar(kBarSFull), G & 1u, 0x30u)) return false;
+    ptx::tc_fence_after();
+    ptx::tmem_ld64(tmem + lane_base + kColS, sv);
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(sh.bar(kBarSFree));
+    return true;
+}
+
+// Softmax of page G of the current item: combines the own partial scores `sv` with the
+// peer's, updates the row state, writes P into TMEM and hands it to the MMA warp.
+__device__ __forceinline__ bool softmax_page(const DecodeParams& p, const Shared& sh, uint32_t tmem,
+                                             uint32_t lane_base, int row,
+                                             const Item& it, int n_vis, uint32_t j, uint32_t G,
+                                             const uint32_t* sv, RowState& st) {
+    const uint32_t xb = G & 1u;
+    if (!warp_wait_bar<true>(sh, sh.bar(kBarXFull + xb), (G >> 1) & 1u, 0x32u)) return false;
+    // s = (own + peer) * scale_log2, peer = (v - 32768) * peer_scale where v is the biased
+    // 16-bit code: 2^23 + v is formed by OR-ing v into the bits of 2^23, and subtracting
+    // 2^23 + 32768 from it is exact, so dequantising rounds only once
+    float s[64];
+    const uint32_t buf = sh.base_u32 + kOffX + xb * kXBytes;
+    float pscale;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(pscale) : "r"(buf + kXDataBytes + 4 * row) : "memory");
+    const float a = pscale * p.scale_log2;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+        ptx::ld_shared_v4(buf + (uint32_t)row * 128 + (uint32_t)((c ^ (row & 7)) * 16), w[0], w[1],
+                          w[2], w[3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(0x4B000000u | (w[e] & 0xffffu));
+            const float hi = __uint_as_float(0x4B000000u | (w[e] >> 16));
+            const int q = 8 * c + 2 * e;
+            s[q] = fmaf(lo - 8421376.f, a, f32(sv[q]) * p.scale_log2);
+            s[q + 1] = fmaf(hi - 8421376.f, a, f32(sv[q + 1]) * p.scale_log2);
+        }
+    }
+    // buffer xb is consumed: tell the senders, and re-arm it for page G + 2 (the peer
+    // cannot send that page before every row here has passed the wait above)
+    ptx::mbar_arrive(sh.bar(kBarXRead + xb));
+    if (row == 0) ptx::mbar_arrive_expect_tx(sh.bar(kBarXFull + xb), kXPayload);
+
+    // mask tokens past this row's visible end
+    const int t0 = (it.k_lo + (int)j) * kBlock;
+    const int lim = n_vis - t0;                        // valid columns: [0, lim)
+    float mx = -INFINITY;
+    if (!__all_sync(0xffffffffu, lim >= 64)) {
+#pragma unroll
+        for (int q = 0; q < 64; ++q) s[q] = q < lim ? s[q] : -INFINITY;
+    }
+    {
+        float m8[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+            m8[a] = fmaxf(fmaxf(fmaxf(s[a], s[a + 8]), fmaxf(s[a + 16], s[a + 24])),
+                          fmaxf(fmaxf(s[a + 32], s[a + 40]), fmaxf(s[a + 48], s[a + 56])));
+        }
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+    }
+    // raise the reference max only when it grows past the threshold
+    const bool raise = mx > st.m_ref + kRescaleLog2 || (st.m_ref == -INFINITY && mx > -INFINITY);
+    float factor = 1.f;
+    if (raise) {
+        factor = st.m_ref == -INFINITY ? 0.f : ptx::ex2_ftz(st.m_ref - mx);
+        st.m_ref = mx;
+        st.l_sum *= factor;
+    }
+    const bool need_o = raise && j > 0 && factor != 1.f;
+    if (__any_sync(0xffffffffu, need_o)) {
+        // O must hold the previous page's PV before it is rescaled
+        if (!warp_wait_bar<false>(sh, sh.bar(kBarPvDone + (xb ^ 1u)), ((G - 1) >> 1) & 1u, 0x33u))
+            return false;
+        ptx::tc_fence_after();
+        const float f = need_o ? factor : 1.f;
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+            uint32_t ov[32];
+            const uint32_t oaddr = tmem + lane_base + kColO + 32 * cc;
+            ptx::tmem_ld32(oaddr, ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(f32(ov[e]) * f);
+            ptx::tmem_st32(oaddr, ov);
+        }
+    }
+    const float mb = st.m_ref == -INFINITY ? 0.f : st.m_ref;
+    uint32_t pk[32];
+    float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+        const float p0 = ptx::ex2_ftz(s[2 * q] - mb);
+        const float p1 = ptx::ex2_ftz(s[2 * q + 1] - mb);
+        rs0 += p0;
+        rs1 += p1;
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        pk[q] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    st.l_sum += rs0 + rs1;
+    // P buffer G % 2 is free once PV of page G - 2 has completed
+    if (G >= 2 && !warp_wait_bar<false>(sh, sh.bar(kBarPvDone + xb), ((G - 2) >> 1) & 1u, 0x35u))
+        return false;
+    ptx::tc_fence_after();
+    ptx::tmem_st32(tmem + lane_base + kColP + 32 * xb, pk);
+
+    // zero V rows past the sequence end on its last, partial page (they may hold stale
+    // or NaN data, and P = 0 would not cancel NaN in the MMA)
+    const int tail = it.L - t0;
+    if (tail < kBlock) {
+        const uint32_t stg = sh.stage(G % kStages);
+        const int nbad = kBlock - tail;
+        for (int q = row; q < nbad * 32; q += 128) {
+            const int rr = tail + (q >> 5);
+            const int box = (q >> 3) & 3;
+            const int ch = q & 7;
+            ptx::st_shared_v4(stg + box * kBoxBytes + rr * 128 + ch * 16, 0, 0, 0, 0);
+        }
+        ptx::fence_proxy_async_smem();
+    }
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(sh.bar(kBarPReady + xb));
+    return true;
+}
 
 __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared& sh, uint32_t tmem,
                                             uint32_t crank, int quarter, int lane) {
     const int row = quarter * 32 + lane;                   // TMEM lane == query row in tile
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const uint32_t peer = crank ^ 1u;
-    const uint32_t xrow_own = sh.base_u32 + kOffX + (uint32_t)row * kXRowStride;
-    const uint32_t xrow_peer = ptx::mapa(xrow_own, peer);
-    const uint32_t xfull_peer = ptx::mapa(sh.bar(kBarXFull), peer);
-    const uint32_t xfree_peer = ptx::mapa(sh.bar(kBarXFree), peer);
-    const int tid = quarter * 32 + lane;                   // 0..127 within the group
 
     ItemIter iter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item it;
     uint32_t G = 0;
-    uint32_t g = 0;
     while (iter.next(it)) {
         const int r = it.t * kTileRows + row;               // query row within the sequence
         const bool row_valid = r < p.rows;
@@ -288,22 +537,22 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
                 p.q + ((size_t)it.b * p.rows + (row_valid ? r : 0)) * kHeadDim);
             const uint32_t qaddr = tmem + lane_base + kColQ;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int cc = 0; cc < 4; ++cc) {
                 uint32_t v[32];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    uint4 x = row_valid ? __ldg(src + crank * 32 + c * 8 + j) : make_uint4(0, 0, 0, 0);
+                    uint4 x = row_valid ? __ldg(src + crank * 32 + cc * 8 + j) : make_uint4(0, 0, 0, 0);
                     v[4 * j + 0] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
                 }
-                ptx::tmem_st32(qaddr + 32 * c, v);
+                ptx::tmem_st32(qaddr + 32 * cc, v);
             }
             // rope half: 32 dims = 4 chunks of 16 B; K-major SW64 layout, 8-row atoms
             const uint32_t qr = sh.base_u32 + kOffQrope + (uint32_t)(row >> 3) * 512 +
                                 (uint32_t)(row & 7) * 64;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint4 x = row_valid ? __ldg(src + 64 + crank * 4 + c) : make_uint4(0, 0, 0, 0);
-                const uint32_t phys = (uint32_t)(c ^ ((row & 7) >> 1));
+            for (int cc = 0; cc < 4; ++cc) {
+                uint4 x = row_valid ? __ldg(src + 64 + crank * 4 + cc) : make_uint4(0, 0, 0, 0);
+                const uint32_t phys = (uint32_t)(cc ^ ((row & 7) >> 1));
                 ptx::st_shared_v4(qr + phys * 16, x.x, x.y, x.z, x.w);
             }
             ptx::fence_proxy_async_smem();
@@ -312,110 +561,20 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
             ptx::mbar_arrive(sh.bar(kBarQReady));
         }
 
-        float m_ref = -INFINITY;      // running reference max (log2 domain)
-        float l_sum = 0.f;
-        const int n = it.k_hi - it.k_lo;
+        RowState st{-INFINITY, 0.f};
+        const uint32_t n = (uint32_t)(it.k_hi - it.k_lo);
+        // page j is finished while page j+1's scores have already been read
+        uint32_t sv[64], sn[64];
+        if (!load_scores(sh, tmem, lane_base, G, sv)) return;
         bool ok = true;
-        for (int j = 0; j < n && ok; ++j, ++G, ++g) {
-            const uint32_t sb = G & 1u;
-            const int k = it.k_lo + j;
-            if (!warp_wait_bar<false>(sh, sh.bar(kBarSFull + sb), (G >> 1) & 1u, 0x30u)) { ok = false; break; }
-            ptx::tc_fence_after();
-            uint32_t sv[64];
-            const uint32_t saddr = tmem + lane_base + kColS + 64 * sb;
-            ptx::tmem_ld64(saddr, sv);
-
-            // exchange partial scores with the peer CTA
-            if (G >= 2 && !warp_wait_bar<true>(sh, sh.bar(kBarXFree + sb), ((G - 2) >> 1) & 1u, 0x31u)) {
+        for (uint32_t j = 0; j < n; ++j, ++G) {
+            if (j + 1 < n && !load_scores(sh, tmem, lane_base, G + 1, sn)) { ok = false; break; }
+            if (!softmax_page(p, sh, tmem, lane_base, row, it, n_vis, j, G, sv, st)) {
                 ok = false;
                 break;
             }
-            const uint32_t dst = xrow_peer + sb * kXBytes;
 #pragma unroll
-            for (int c = 0; c < 16; ++c)
-                ptx::st_cluster_v4(dst + 16 * c, sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
-            ptx::mbar_arrive_remote(xfull_peer + 8 * sb);
-            if (!warp_wait_bar<true>(sh, sh.bar(kBarXFull + sb), (G >> 1) & 1u, 0x32u)) { ok = false; break; }
-            float s[64];
-            const uint32_t src = xrow_own + sb * kXBytes;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                uint32_t a, b2, c2, d;
-                ptx::ld_shared_v4(src + 16 * c, a, b2, c2, d);
-                s[4 * c + 0] = f32(sv[4 * c + 0]) + f32(a);
-                s[4 * c + 1] = f32(sv[4 * c + 1]) + f32(b2);
-                s[4 * c + 2] = f32(sv[4 * c + 2]) + f32(c2);
-                s[4 * c + 3] = f32(sv[4 * c + 3]) + f32(d);
-            }
-            ptx::mbar_arrive_remote(xfree_peer + 8 * sb);
-
-            // scale into the log2 domain and mask tokens past this row's visible end
-            const int t0 = k * kBlock;
-            const int lim = n_vis - t0;                      // valid columns: [0, lim)
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                s[c] = c < lim ? s[c] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[c]);
-            }
-            // raise the reference max only when it grows past the threshold
-            const bool raise = mx > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mx > -INFINITY);
-            float factor = 1.f;
-            if (raise) {
-                factor = m_ref == -INFINITY ? 0.f : exp2f(m_ref - mx);
-                m_ref = mx;
-                l_sum *= factor;
-            }
-            const bool need_o = raise && j > 0 && factor != 1.f;
-            if (__any_sync(0xffffffffu, need_o)) {
-                // O must hold the previous page's PV before it is rescaled
-                if (!warp_wait_bar<false>(sh, sh.bar(kBarPvDone + (sb ^ 1u)), ((G - 1) >> 1) & 1u, 0x33u)) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-                const float f = need_o ? factor : 1.f;
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t ov[32];
-                    const uint32_t oaddr = tmem + lane_base + kColO + 32 * c;
-                    ptx::tmem_ld32(oaddr, ov);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(f32(ov[e]) * f);
-                    ptx::tmem_st32(oaddr, ov);
-                }
-            }
-            const float mb = m_ref == -INFINITY ? 0.f : m_ref;
-            uint32_t pk[32];
-            float rs = 0.f;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float p0 = exp2f(s[2 * c] - mb);
-                const float p1 = exp2f(s[2 * c + 1] - mb);
-                rs += p0 + p1;
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                pk[c] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            l_sum += rs;
-            ptx::tmem_st32(saddr, pk);
-
-            // zero V rows past the sequence end on its last, partial page (they may
-            // hold stale or NaN data and P = 0 would not cancel NaN in the MMA)
-            const int tail = it.L - t0;
-            if (tail < kBlock) {
-                const uint32_t st = sh.stage(g % kStages);
-                const int nbad = kBlock - tail;
-                for (int c = tid; c < nbad * 32; c += 128) {
-                    const int rr = tail + (c >> 5);
-                    const int box = (c >> 3) & 3;
-                    const int ch = c & 7;
-                    ptx::st_shared_v4(st + box * kBoxBytes + rr * 128 + ch * 16, 0, 0, 0, 0);
-                }
-                ptx::fence_proxy_async_smem();
-            }
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(sh.bar(kBarPReady + sb));
+            for (int q = 0; q < 64; ++q) sv[q] = sn[q];
         }
         if (!ok) return;
 
@@ -423,18 +582,19 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
         const uint32_t Gl = G - 1;
         if (!warp_wait_bar<false>(sh, sh.bar(kBarPvDone + (Gl & 1u)), (Gl >> 1) & 1u, 0x34u)) return;
         ptx::tc_fence_after();
-        const bool empty = !(l_sum > 0.f);
-        const float inv = empty ? 0.f : 1.f / l_sum;
-        const float lse2 = empty ? -INFINITY : m_ref + __log2f(l_sum);
+        const bool empty = !(st.l_sum > 0.f);
+        const float inv = empty ? 0.f : 1.f / st.l_sum;
+        const float lse2 = empty ? -INFINITY : st.m_ref + __log2f(st.l_sum);
         const bool final_out = it.n_chunks == 1;
         const bool have_ws = it.part < p.max_chunks;
-        if (!final_out && !have_ws && tid == 0) record_error(kErrWorkspace, (uint32_t)it.v & 0xffffffu);
+        if (!final_out && !have_ws && row == 0)
+            record_error(kErrWorkspace, (uint32_t)it.v & 0xffffffu);
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int cc = 0; cc < 8; ++cc) {
             uint32_t ov[32];
-            ptx::tmem_ld32(tmem + lane_base + kColO + 32 * c, ov);
+            ptx::tmem_ld32(tmem + lane_base + kColO + 32 * cc, ov);
             if (!row_valid) continue;
-            const int col = (int)crank * kLatentHalf + 32 * c;
+            const int col = (int)crank * kLatentHalf + 32 * cc;
             if (final_out) {
                 uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)it.b * p.rows + r) * kHeadDimV + col);
 #pragma unroll
@@ -488,41 +648,51 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_lat,
             ptx::mbar_init(sh.bar(kBarFull + s), 1);
             ptx::mbar_init(sh.bar(kBarEmpty + s), 1);
         }
+        ptx::mbar_init(sh.bar(kBarSFull), 1);
+        ptx::mbar_init(sh.bar(kBarSFree), 256);
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(sh.bar(kBarSFull + i), 1);
             ptx::mbar_init(sh.bar(kBarPReady + i), 128);
             ptx::mbar_init(sh.bar(kBarPvDone + i), 1);
-            ptx::mbar_init(sh.bar(kBarXFull + i), 128);
-            ptx::mbar_init(sh.bar(kBarXFree + i), 128);
+            ptx::mbar_init(sh.bar(kBarXFull + i), 1);
+            ptx::mbar_init(sh.bar(kBarXRead + i), 128);
+            ptx::mbar_init(sh.bar(kBarXFree + i), 1);
+            ptx::mbar_init(sh.bar(kBarStage + i), 128);
         }
         ptx::mbar_init(sh.bar(kBarQReady), 128);
         *sh.abort_flag() = 0;
         ptx::fence_mbarrier_init_cluster();
+        // arm both exchange buffers for the first two pages
+        ptx::mbar_arrive_expect_tx(sh.bar(kBarXFull + 0), kXPayload);
+        ptx::mbar_arrive_expect_tx(sh.bar(kBarXFull + 1), kXPayload);
         ptx::prefetch_tensormap(&tm_lat);
         ptx::prefetch_tensormap(&tm_rope);
     }
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         ptx::tmem_alloc(ptx::smem_u32(sh.tmem_slot()), kTmemCols);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
     __syncthreads();
-    ptx::cluster_sync();            // peer barriers initialised before any remote arrive
+    ptx::cluster_sync();            // peer barriers initialised before any remote access
     ptx::tc_fence_after();
     const uint32_t tmem = *sh.tmem_slot();
 
-    if (warp == 0) {
-        if (lane == 0) run_producer(p, sh, &tm_lat, &tm_rope, crank);
-    } else if (warp == 1) {
-        if (lane == 0) run_mma(p, sh, tmem);
+    if (warp < kWarpSender0) {
+        ptx::setmaxnreg_inc<kRegsSoftmax>();
+        run_softmax(p, sh, tmem, crank, warp, lane);
+    } else if (warp < kWarpProducer) {
+        ptx::setmaxnreg_dec<kRegsSender>();
+        run_sender(p, sh, tmem, crank, warp - kWarpSender0, lane);
     } else {
-        run_softmax(p, sh, tmem, crank, warp & 3, lane);
+        ptx::setmaxnreg_dec<kRegsControl>();
+        if (warp == kWarpProducer && lane == 0) run_producer(p, sh, &tm_lat, &tm_rope, crank);
+        if (warp == kWarpMma && lane == 0) run_mma(p, sh, tmem);
     }
 
     ptx::tc_fence_before();
     __syncthreads();
     ptx::cluster_sync();            // no remote store or arrive may target an exited CTA
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }

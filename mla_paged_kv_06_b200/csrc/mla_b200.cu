@@ -58,6 +58,13 @@ bool prepare_sm100_kernel(int dev) {
     if (cudaFuncSetAttribute(sm100::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sm100::kSmemAlloc) != cudaSuccess)
         return false;
+    // The warpgroups raise and lower their register budgets at start; the raised sum must
+    // fit in what the CTA is launched with, or the raising warpgroup would wait forever.
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, sm100::decode_kernel) != cudaSuccess) return false;
+    const long pool = (long)attr.numRegs * sm100::kThreads;
+    const long need = 128L * (sm100::kRegsSoftmax + sm100::kRegsSender + sm100::kRegsControl);
+    if (pool < need || attr.maxThreadsPerBlock < sm100::kThreads) return false;
     done[dev] = 1;
     return true;
 }
