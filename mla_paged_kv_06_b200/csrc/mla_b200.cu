@@ -63,7 +63,7 @@ bool prepare_sm100_kernel(int dev) {
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, sm100::decode_kernel) != cudaSuccess) return false;
     const long pool = (long)attr.numRegs * sm100::kThreads;
-    const long need = 128L * (sm100::kRegsSoftmax + sm100::kRegsSender + sm100::kRegsControl);
+    const long need = (long)sm100::kRegsNeeded;
     if (pool < need || attr.maxThreadsPerBlock < sm100::kThreads) return false;
     done[dev] = 1;
     return true;
