@@ -32,6 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from mla_paged_kv_06_b200 import workloads as wl  # noqa: E402
+from mla_paged_kv_06_b200.shard import max_over_ranks, rank_seed  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
 LAUNCHES_PER_STEP = 3               # metadata, split kernel, combine kernel
@@ -221,7 +222,7 @@ def main():
     from mla_paged_kv_06_b200 import mla
 
     # each rank decodes its own batch of the same shape (weak scaling)
-    x = wl.make_workload(args.workload, seed=args.seed + rank)
+    x = wl.make_workload(args.workload, seed=rank_seed(args.seed, rank))
     d = dict(q=x.q.cuda(), kcache=x.kcache.cuda(), block_table=x.block_table.cuda(),
              seqlens=x.seqlens.cuda())
     nsm = mla.default_num_sms()
@@ -271,11 +272,7 @@ def main():
     step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
     decode_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
     meta_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error during timing: {mla.status_string(st)} {word:#x}")
@@ -310,10 +307,7 @@ def main():
         b.record(stream)
         b.synchronize()
         e2e_ms += a.elapsed_time(b)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
 
     hbm_peak, tf_peak, peak_kind = peaks()
     avg_decode_s = statistics.mean(decode_ms) / 1e3
