@@ -32,7 +32,8 @@
  *
  * Asynchrony: mla_get_metadata and mla_decode_fwd only enqueue work on `stream`
  * (a cudaStream_t passed as void*; NULL is the legacy default stream) and never
- * synchronise, so both can be captured in a CUDA graph.
+ * synchronise it. The first mla_decode_fwd on a device also sets the kernel's
+ * shared-memory limit and queries its cluster occupancy once (cached afterwards).
  *
  * Errors: every call checks its arguments on the host first and returns a negative
  * mla_status without launching anything when they are invalid. A launch failure is
