@@ -78,6 +78,7 @@ typedef int mla_status;
 #define MLA_MAX_ROWS       1024   /* s_q * h_q                                        */
 #define MLA_MAX_BATCH     65536
 #define MLA_METADATA_INTS_PER_UNIT 8
+#define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)  /* scratch of mla_decode_fwd_noalloc */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* mla_status_string(mla_status status);
@@ -144,6 +145,43 @@ mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blo
                           const int32_t* metadata, const int32_t* num_splits,
                           void* workspace, size_t workspace_bytes,
                           uint16_t* out, float* lse, void* stream);
+
+/*
+ * mla_decode_fwd without a workspace argument, for callers that cannot hand the
+ * library a scratch buffer. Examples are a serving runtime whose device memory is laid
+ * out once at start-up and may not grow between decode steps, and a caller whose
+ * allocator cannot give out temporary blocks on the decode path (an allocation there
+ * may synchronise the device or fragment a pre-planned pool). The pages describe no
+ * such call: FlashMLA's own interface is not given there, so this has no counterpart
+ * in them and is an addition of this library.
+ *
+ * Arguments, layouts, results and errors are those of mla_decode_fwd, minus
+ * `workspace` and `workspace_bytes`. The split partials go to a scratch array of
+ * MLA_NOALLOC_SCRATCH_BYTES (64 MiB) that lives inside the library as static device
+ * memory, one copy per device, created when the library's kernels are loaded there.
+ * Neither this call nor its set-up allocates device or host memory.
+ *
+ *   Limit: sizes whose worst-case partials exceed the array, over every schedule the
+ *     current device can run (one [128][512] fp32 tile per work sequence plus one per
+ *     work unit), return MLA_ERR_WORKSPACE_TOO_SMALL before anything is launched. On a
+ *     148-SM B200 that admits batch * ceil(s_q*h_q/128) up to 181. Larger batches must
+ *     use mla_decode_fwd with a workspace.
+ *   First call: the first call on each device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress) and does mla_decode_fwd's one-time
+ *     kernel set-up. Make that first call before any stream capture begins.
+ *   Sharing: every call on a device, from any stream or host thread, uses the same
+ *     array, which keeps the partials of the last call. Nothing in it has to start at
+ *     zero: a call reads only partials it has written itself.
+ *   Races: calls whose GPU work can overlap (different streams with no ordering between
+ *     them, or host threads launching on unsynchronised streams) write the same array
+ *     and corrupt each other's results. Order them on one stream or with events.
+ */
+mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                                  const int32_t* block_table, int max_blocks,
+                                  const int32_t* seqlens, int batch, int s_q, int h_q,
+                                  float scale, int causal,
+                                  const int32_t* metadata, const int32_t* num_splits,
+                                  uint16_t* out, float* lse, void* stream);
 
 /*
  * Reads and clears the device-side error word of the current device after

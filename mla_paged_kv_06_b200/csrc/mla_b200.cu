@@ -18,6 +18,11 @@
 #include "metadata.cuh"
 #include "sched.cuh"
 
+// Split-partial scratch of mla_decode_fwd_noalloc: a fixed array inside the library in
+// place of a caller-provided workspace. One copy exists per device; every call of that
+// entry point on the device shares it (see include/mla.h for the rules that follow).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 using namespace mla;
@@ -192,6 +197,24 @@ DecodeParams make_params(const uint16_t* q, const uint16_t* kcache, int num_bloc
     return p;
 }
 
+// Device address of g_noalloc_scratch on `dev`, which must be the current device. Looked
+// up on the first call for each device and cached; nullptr if the lookup fails.
+void* noalloc_scratch(int dev) {
+    static std::mutex mu;
+    static std::vector<void*> addr;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)addr.size() <= dev) addr.resize(dev + 1, nullptr);
+    if (!addr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = ptr;
+    }
+    return addr[dev];
+}
+
 mla_status launch_combine(const DecodeParams& p, cudaStream_t s) {
     dim3 grid(p.batch * p.tiles, kTileRows / kCombineRowsPerCta);
     combine_kernel<<<grid, kCombineThreads, 0, s>>>(p);
@@ -292,6 +315,40 @@ mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blo
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
     const int pairs = device_pairs(dev);
     if (pairs < 1 || !prepare_sm100_kernel(dev)) return MLA_ERR_CUDA;
+    CUtensorMap tm_lat, tm_rope;
+    if (!make_pool_map(&tm_lat, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_pool_map(&tm_rope, kcache, num_blocks, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+        return MLA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    sm100::decode_kernel<<<2 * pairs, sm100::kThreads, sm100::kSmemAlloc, s>>>(p, tm_lat, tm_rope);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    return launch_combine(p, s);
+}
+
+mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                                  const int32_t* block_table, int max_blocks,
+                                  const int32_t* seqlens, int batch, int s_q, int h_q,
+                                  float scale, int causal, const int32_t* metadata,
+                                  const int32_t* num_splits, uint16_t* out, float* lse,
+                                  void* stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    void* scratch = noalloc_scratch(dev);
+    if (!scratch) return MLA_ERR_CUDA;
+    const size_t scratch_bytes = MLA_NOALLOC_SCRATCH_BYTES;
+    mla_status st = validate_decode(q, kcache, num_blocks, block_table, max_blocks, seqlens,
+                                    batch, s_q, h_q, scale, causal, metadata, num_splits,
+                                    scratch, scratch_bytes, out, lse);
+    if (st != MLA_OK) return st;
+    const int pairs = device_pairs(dev);
+    if (pairs < 1 || !prepare_sm100_kernel(dev)) return MLA_ERR_CUDA;
+    // worst case over every schedule this device can run: one chunk per work sequence
+    // plus one per unit
+    if (mla_workspace_bytes(batch, h_q, s_q, 2 * pairs) > scratch_bytes)
+        return MLA_ERR_WORKSPACE_TOO_SMALL;
+    DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
+                                 batch, s_q, h_q, scale, causal, metadata, num_splits,
+                                 scratch, scratch_bytes, out, lse);
     CUtensorMap tm_lat, tm_rope;
     if (!make_pool_map(&tm_lat, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_pool_map(&tm_rope, kcache, num_blocks, 32, CU_TENSOR_MAP_SWIZZLE_64B))

@@ -25,6 +25,7 @@ MLA_ERR_CUDA = -3
 MLA_ERR_WORKSPACE_TOO_SMALL = -4
 MLA_ERR_DEVICE_TIMEOUT = -5
 MLA_ERR_DEVICE_BAD_INPUT = -6
+MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class MlaError(RuntimeError):
@@ -50,6 +51,8 @@ def _load() -> ctypes.CDLL:
                                  vp, vp, vp, sz, vp, vp, vp]),
         "mla_decode_fwd_simt": (i32, [vp, vp, i32, vp, i32, vp, i32, i32, i32, f32, i32,
                                       vp, vp, vp, sz, vp, vp, vp]),
+        "mla_decode_fwd_noalloc": (i32, [vp, vp, i32, vp, i32, vp, i32, i32, i32, f32, i32,
+                                         vp, vp, vp, vp, vp]),
         "mla_get_last_device_error": (i32, [vp, ctypes.POINTER(ctypes.c_uint32)]),
         "mla_plan_host": (i32, [vp, i32, i32, i32, i32, vp, vp]),
     }
@@ -174,6 +177,25 @@ def mla_decode_fwd_simt(q, kcache, block_table, seqlens, scale, causal, metadata
     """Same as mla_decode_fwd on the CUDA-core kernel."""
     return _decode("mla_decode_fwd_simt", q, kcache, block_table, seqlens, scale, causal,
                    metadata, num_splits, workspace, out, lse, stream, num_sms)
+
+
+def mla_decode_fwd_noalloc(q, kcache, block_table, seqlens, scale, causal, metadata,
+                           num_splits, out=None, lse=None, stream=None):
+    """mla_decode_fwd with the library's built-in scratch instead of a workspace (the C
+    call allocates nothing; `out` and `lse` are created here when not given)."""
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 4 and q.is_contiguous()
+    assert kcache.dtype == torch.bfloat16 and kcache.is_contiguous()
+    assert block_table.dtype == torch.int32 and block_table.is_contiguous()
+    batch, s_q, h_q, _ = q.shape
+    if out is None:
+        out = torch.empty((batch, s_q, h_q, 512), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((batch, h_q, s_q), dtype=torch.float32, device=q.device)
+    _check(_lib.mla_decode_fwd_noalloc(
+        _ptr(q), _ptr(kcache), kcache.shape[0], _ptr(block_table), block_table.shape[1],
+        _ptr(seqlens), batch, s_q, h_q, float(scale), int(bool(causal)), _ptr(metadata),
+        _ptr(num_splits), _ptr(out), _ptr(lse), _stream(stream)), "mla_decode_fwd_noalloc")
+    return out, lse
 
 
 def mla_get_last_device_error(stream=None):
