@@ -261,7 +261,7 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
     uint32_t idle = 0;
     for (;;) {
         if (gv < gq && (gv < (uint32_t)kVStages ||
-                        ptx::mbar_try_wait(sh.bar(kBarVEmpty + gv % kVStages),
+                        ptx::mbar_test_wait(sh.bar(kBarVEmpty + gv % kVStages),
                                            ((gv / kVStages) - 1) & 1u))) {
             const uint32_t full = sh.bar(kBarVFull + gv % kVStages);
             ptx::mbar_arrive_expect_tx(full, kVStageBytes);
@@ -274,7 +274,7 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             idle = 0;
         } else if (have && gq < gv + kPidRing &&
                    (gq < (uint32_t)kQkStages ||
-                    ptx::mbar_try_wait(sh.bar(kBarQkEmpty + gq % kQkStages),
+                    ptx::mbar_test_wait(sh.bar(kBarQkEmpty + gq % kQkStages),
                                        ((gq / kQkStages) - 1) & 1u))) {
             int pid = p.block_table[(size_t)it.b * p.max_blocks + k];
             if (pid < 0 || pid >= p.num_blocks) {
@@ -324,14 +324,14 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
 // ------------------------------------------------------------------ MMA issuer (warp 9)
 // QK of page G may start once its page has landed and the senders have read S of G - 1.
 __device__ __forceinline__ bool qk_ready(const Shared& sh, uint32_t G) {
-    return ptx::mbar_try_wait(sh.bar(kBarQkFull + G % kQkStages), (G / kQkStages) & 1u) &&
-           (G == 0 || ptx::mbar_try_wait(sh.bar(kBarSFree), (G - 1) & 1u));
+    return ptx::mbar_test_wait(sh.bar(kBarQkFull + G % kQkStages), (G / kQkStages) & 1u) &&
+           (G == 0 || ptx::mbar_test_wait(sh.bar(kBarSFree), (G - 1) & 1u));
 }
 
 // PV of page G may start once its P is in TMEM and its latent dims are in the V ring.
 __device__ __forceinline__ bool pv_ready(const Shared& sh, uint32_t G) {
-    return ptx::mbar_try_wait(sh.bar(kBarPReady + (G & 1u)), (G >> 1) & 1u) &&
-           ptx::mbar_try_wait(sh.bar(kBarVFull + G % kVStages), (G / kVStages) & 1u);
+    return ptx::mbar_test_wait(sh.bar(kBarPReady + (G & 1u)), (G >> 1) & 1u) &&
+           ptx::mbar_test_wait(sh.bar(kBarVFull + G % kVStages), (G / kVStages) & 1u);
 }
 
 // S = Q K^T for global page index G (QK stage G % kQkStages); qk_ready(G) has been seen.

@@ -14,7 +14,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "decode_simt.cuh"
-#include "decode_sm100.cuh"
+#include "decode_pair.cuh"
 #include "metadata.cuh"
 #include "sched.cuh"
 
@@ -54,22 +54,18 @@ size_t ws_capacity(size_t bytes) {
 size_t ws_o_offset(size_t cap) { return align_up(kWsHeader + cap * kTileRows * 4, kAlign); }
 
 // Opt the split kernel into its shared-memory footprint (once per device).
-bool prepare_sm100_kernel(int dev) {
+bool prepare_split_kernel(int dev) {
     static std::mutex mu;
     static std::vector<char> done;
     std::lock_guard<std::mutex> lock(mu);
     if ((int)done.size() <= dev) done.resize(dev + 1, 0);
     if (done[dev]) return true;
-    if (cudaFuncSetAttribute(sm100::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sm100::kSmemAlloc) != cudaSuccess)
+    if (cudaFuncSetAttribute(pair::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)pair::kSmemAlloc) != cudaSuccess)
         return false;
-    // The warpgroups raise and lower their register budgets at start; the raised sum must
-    // fit in what the CTA is launched with, or the raising warpgroup would wait forever.
     cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, sm100::decode_kernel) != cudaSuccess) return false;
-    const long pool = (long)attr.numRegs * sm100::kThreads;
-    const long need = (long)sm100::kRegsNeeded;
-    if (pool < need || attr.maxThreadsPerBlock < sm100::kThreads) return false;
+    if (cudaFuncGetAttributes(&attr, pair::decode_kernel) != cudaSuccess) return false;
+    if (attr.maxThreadsPerBlock < pair::kThreads) return false;
     done[dev] = 1;
     return true;
 }
@@ -87,11 +83,11 @@ int device_pairs(int dev) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return -1;
     int pairs = sms / 2 < 1 ? 1 : sms / 2;
-    if (prepare_sm100_kernel(dev)) {
+    if (prepare_split_kernel(dev)) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * pairs);
-        cfg.blockDim = dim3(sm100::kThreads);
-        cfg.dynamicSmemBytes = sm100::kSmemAlloc;
+        cfg.blockDim = dim3(pair::kThreads);
+        cfg.dynamicSmemBytes = pair::kSmemAlloc;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -100,7 +96,7 @@ int device_pairs(int dev) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, sm100::decode_kernel, &cfg) == cudaSuccess &&
+        if (cudaOccupancyMaxActiveClusters(&clusters, pair::decode_kernel, &cfg) == cudaSuccess &&
             clusters > 0 && clusters < pairs)
             pairs = clusters;
         cudaGetLastError();
@@ -314,13 +310,11 @@ mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blo
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
     const int pairs = device_pairs(dev);
-    if (pairs < 1 || !prepare_sm100_kernel(dev)) return MLA_ERR_CUDA;
-    CUtensorMap tm_lat, tm_rope;
-    if (!make_pool_map(&tm_lat, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_pool_map(&tm_rope, kcache, num_blocks, 32, CU_TENSOR_MAP_SWIZZLE_64B))
-        return MLA_ERR_CUDA;
+    if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
+    CUtensorMap tm;
+    if (!make_pool_map(&tm, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    sm100::decode_kernel<<<2 * pairs, sm100::kThreads, sm100::kSmemAlloc, s>>>(p, tm_lat, tm_rope);
+    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return launch_combine(p, s);
 }
@@ -341,7 +335,7 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
                                     scratch, scratch_bytes, out, lse);
     if (st != MLA_OK) return st;
     const int pairs = device_pairs(dev);
-    if (pairs < 1 || !prepare_sm100_kernel(dev)) return MLA_ERR_CUDA;
+    if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
     // worst case over every schedule this device can run: one chunk per work sequence
     // plus one per unit
     if (mla_workspace_bytes(batch, h_q, s_q, 2 * pairs) > scratch_bytes)
@@ -349,12 +343,10 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
     DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
                                  batch, s_q, h_q, scale, causal, metadata, num_splits,
                                  scratch, scratch_bytes, out, lse);
-    CUtensorMap tm_lat, tm_rope;
-    if (!make_pool_map(&tm_lat, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_pool_map(&tm_rope, kcache, num_blocks, 32, CU_TENSOR_MAP_SWIZZLE_64B))
-        return MLA_ERR_CUDA;
+    CUtensorMap tm;
+    if (!make_pool_map(&tm, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    sm100::decode_kernel<<<2 * pairs, sm100::kThreads, sm100::kSmemAlloc, s>>>(p, tm_lat, tm_rope);
+    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return launch_combine(p, s);
 }
