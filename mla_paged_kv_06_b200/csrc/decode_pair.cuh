@@ -34,6 +34,10 @@
 //   warp 8    TMA producer: whole pages into a 2-stage ring (the stage frees when PV of
 //             its step is done), the post-QK reloads, and L2 prefetch of pages ahead.
 //   warp 9    TMEM owner (both CTAs) and, in CTA 0, the MMA issuer.
+// CTA 1's warps tell CTA 0's barriers that their Q or P is ready with a 4-byte
+// asynchronous store whose completion counts bytes on the barrier (release at cluster
+// scope without stalling the warp; a remote mbarrier arrive stalls its thread for over
+// a thousand cycles). CTA 0's MMA thread arms those barriers with the bytes to expect.
 // Shared memory: 2 stages x 9 boxes (64 tokens x 64 dims, 128-byte swizzle), Q's upper
 // 320 dims (5 boxes), 2 P buffers (64 rows x 128 tokens), small exchange arrays.
 // TMEM columns: O [0,256) fp32, Q lower latent [256,384) bf16x2 (the 2-CTA A-from-TMEM
@@ -84,7 +88,10 @@ enum : uint32_t {
     kBarDrain = kBarLsum + 1,       // the MMA issuer's last commit
     kNumBars = kBarDrain + 1
 };
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort flag
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort flag, sink word
+// bytes CTA 1 signals per phase: one 4-byte store per softmax warp that arrives
+constexpr uint32_t kPReadyTx = 4 * 4;
+constexpr uint32_t kQReadyTx = 8 * 4;
 constexpr uint32_t kSmemBytes = kOffMisc + 16;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;      // room to align the base to 1 KB
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
@@ -108,6 +115,7 @@ struct Shared {
         return reinterpret_cast<volatile int*>(base + kOffMisc + 8);
     }
     __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + kOffMisc); }
+    __device__ uint32_t sink() const { return base_u32 + kOffMisc + 12; }
 };
 
 // Bounded wait (as in every kernel of the library): false if the phase does not complete
@@ -342,6 +350,7 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Shared& sh,
     uint32_t items = 0;
     while (iter.next(it)) {
         if (!wait_bar<true>(sh, sh.bar(kBarQReady), items & 1u, 0x20u)) break;
+        ptx::mbar_arrive_expect_tx(sh.bar(kBarQReady), kQReadyTx);      // the next item's
         ptx::tc_fence_after();
         const uint32_t n = (uint32_t)it.steps();
         uint32_t qk = 0, pv = 0;
@@ -353,6 +362,7 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Shared& sh,
             if (pv < qk &&
                 ptx::mbar_test_wait_cluster(sh.bar(kBarPReady + (Sv & 1u)), (Sv >> 1) & 1u)) {
                 issue_pv(sh, tmem, Sv, pv == 0);
+                ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + (Sv & 1u)), kPReadyTx);  // step Sv+2
                 ++pv;
                 idle = 0;
             } else if (qk < n && qk < pv + 2 &&
@@ -535,8 +545,10 @@ __device__ __forceinline__ bool softmax_step(const DecodeParams& p, const Shared
     ptx::fence_proxy_async_smem();            // P and zeroed rows visible to the MMA
     ptx::tc_fence_before();                   // S read before QK of step S+2 overwrites it
     __syncwarp();
-    if ((threadIdx.x & 31) == 0)
-        ptx::mbar_arrive_remote(ptx::mapa(sh.bar(kBarPReady + b), 0));
+    if ((threadIdx.x & 31) == 0) {
+        if (c.crank == 0) ptx::mbar_arrive(sh.bar(kBarPReady + b));
+        else ptx::st_async_signal(ptx::mapa(sh.sink(), 0), ptx::mapa(sh.bar(kBarPReady + b), 0));
+    }
     return true;
 }
 
@@ -551,7 +563,6 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
     c.half = q >> 1;
     c.grp = warp >> 2;
     const int row = c.row;
-    const uint32_t qready_leader = ptx::mapa(sh.bar(kBarQReady), 0);
 
     ItemIter iter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item it;
@@ -594,7 +605,10 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_remote(qready_leader);
+            if (lane == 0) {
+                if (crank == 0) ptx::mbar_arrive(sh.bar(kBarQReady));
+                else ptx::st_async_signal(ptx::mapa(sh.sink(), 0), ptx::mapa(sh.bar(kBarQReady), 0));
+            }
         }
 
         RowState st{-INFINITY, 0.f};
@@ -687,16 +701,20 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm) {
             ptx::mbar_init(sh.bar(kBarKFull + i), 1);
             ptx::mbar_init(sh.bar(kBarQkDone + i), 1);
             ptx::mbar_init(sh.bar(kBarVFull + i), 1);
-            ptx::mbar_init(sh.bar(kBarPReady + i), 2 * 4);
+            ptx::mbar_init(sh.bar(kBarPReady + i), 4 + 1);      // CTA 0's warps + arming
             ptx::mbar_init(sh.bar(kBarPvDone + i), 1);
             ptx::mbar_init(sh.bar(kBarMaxX + i), 128);
             ptx::mbar_init(sh.bar(kBarMref + i), 128);
         }
-        ptx::mbar_init(sh.bar(kBarQReady), 2 * 8);
+        ptx::mbar_init(sh.bar(kBarQReady), 8 + 1);              // CTA 0's warps + arming
         ptx::mbar_init(sh.bar(kBarLsum), kSoftmaxThreads);
         ptx::mbar_init(sh.bar(kBarDrain), 1);
         *sh.abort_flag() = 0;
         ptx::fence_mbarrier_init_cluster();
+        // arm the first phases of the barriers CTA 1 signals with byte counts
+        ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + 0), kPReadyTx);
+        ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + 1), kPReadyTx);
+        ptx::mbar_arrive_expect_tx(sh.bar(kBarQReady), kQReadyTx);
         ptx::prefetch_tensormap(&tm);
     }
     if (warp == kWarpMma) {

@@ -77,6 +77,17 @@ __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t pa
     return ok != 0;
 }
 
+// Signal a barrier of another CTA without stalling: a 4-byte asynchronous store into
+// that CTA's shared memory (`cluster_addr`, contents irrelevant) whose completion counts 4
+// transaction bytes on its barrier `cluster_bar`. The store is weak, and its complete_tx
+// has release semantics at cluster scope, so this thread's earlier shared-memory writes
+// (and those it has acquired) are visible to whoever observes the barrier's phase.
+__device__ __forceinline__ void st_async_signal(uint32_t cluster_addr, uint32_t cluster_bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+        ::"r"(cluster_addr), "r"(1u), "r"(cluster_bar) : "memory");
+}
+
 // Acquire at cluster scope: pairs with mbar_arrive_remote from the peer CTA.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
     uint32_t ok;
