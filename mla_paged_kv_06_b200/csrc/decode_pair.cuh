@@ -33,6 +33,10 @@
 //             P (bf16) goes to shared memory as the A operand of PV.
 //   warp 8    TMA producer: whole pages into a 2-stage ring (the stage frees when PV of
 //             its step is done), the post-QK reloads, and L2 prefetch of pages ahead.
+//             The pool is seen as a 3-D tensor {64 elements, rows, 9 chunks of 128 B}, so
+//             one instruction lands a page as its 9 swizzled tiles (the TMA unit streams
+//             8 KB boxes at barely half the rate of whole pages) and a reload is two
+//             2-tile instructions.
 //   warp 9    TMEM owner (both CTAs) and, in CTA 0, the MMA issuer.
 // CTA 1's warps tell CTA 0's barriers that their Q or P is ready with a 4-byte
 // asynchronous store whose completion counts bytes on the barrier (release at cluster
@@ -208,13 +212,15 @@ __device__ __forceinline__ int page_row(const DecodeParams& p, int b, int k, int
 }
 
 // ------------------------------------------------------------------ producer (warp 8)
+// tm_page: box {64, 64 rows, 9 chunks} (a whole page); tm_pair: box {64, 64 rows, 2}.
 // Step S uses stage S % 2. This CTA's page of the step is loaded whole once PV of step
 // S - 2 has freed the stage; both CTAs' loads complete on CTA 0's barrier. Once QK of
 // the step is done, the other page's share of this CTA's PV dims is reloaded into the
 // four boxes that only QK needed (CTA 0: boxes 2,3,6,7 <- page B's 0,1,4,5; CTA 1: boxes
 // 0,1,4,5 <- page A's 2,3,6,7), completing on this CTA's own barrier.
 __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared& sh,
-                                             const CUtensorMap* tm, uint32_t crank) {
+                                             const CUtensorMap* tm_page,
+                                             const CUtensorMap* tm_pair, uint32_t crank) {
     ItemIter iter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item it;
     bool have = iter.next(it);
@@ -228,8 +234,7 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
         const int k = pit.k_lo + 2 * pj + (int)crank;
         if (k < pit.k_hi) {
             const int pid = p.block_table[(size_t)pit.b * p.max_blocks + k];
-            if (pid >= 0 && pid < p.num_blocks)
-                for (int i = 0; i < kBoxesPerPage; ++i) ptx::tma_prefetch_2d(tm, 64 * i, pid * kBlock);
+            if (pid >= 0 && pid < p.num_blocks) ptx::tma_prefetch_3d(tm_page, 0, pid * kBlock, 0);
         }
         if (++pj >= pit.steps()) {
             phave = piter.next(pit);
@@ -249,12 +254,12 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             const uint32_t st = sh.stage(gv & 1u);
             const int y = reload_row[gv & 3u];
             // CTA 0 fills boxes 2,3,6,7 from page B's 0,1,4,5; CTA 1 fills 0,1,4,5 from
-            // page A's 2,3,6,7
+            // page A's 2,3,6,7 (two boxes per instruction)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int src = (i & 1) + 4 * (i >> 1) + 2 * (int)crank;   // 0,1,4,5 (+2)
-                const int dst = (i & 1) + 4 * (i >> 1) + 2 * (int)(crank ^ 1u);
-                ptx::tma_load_2d(st + dst * kBoxBytes, tm, full, 64 * src, y);
+            for (int i = 0; i < 2; ++i) {
+                const int src = 4 * i + 2 * (int)crank;                     // 0,4 (+2)
+                const int dst = 4 * i + 2 * (int)(crank ^ 1u);
+                ptx::tma_load_3d(st + dst * kBoxBytes, tm_pair, full, 0, y, src);
             }
             ++gv;
             idle = 0;
@@ -266,10 +271,7 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             reload_row[gk & 3u] = page_row(p, it.b, ka + (int)(crank ^ 1u), it.k_hi);
             if (crank == 0) ptx::mbar_arrive_expect_tx(sh.bar(kBarKFull + (gk & 1u)), 2 * kPageBytes);
             const uint32_t st = sh.stage(gk & 1u);
-#pragma unroll
-            for (int i = 0; i < kBoxesPerPage; ++i)
-                ptx::tma_load_2d_pair(st + i * kBoxBytes, tm, kfull_leader + 8 * (gk & 1u),
-                                      64 * i, own);
+            ptx::tma_load_3d_pair(st, tm_page, kfull_leader + 8 * (gk & 1u), 0, own, 0);
             prefetch_next();
             ++gk;
             if (++j >= it.steps()) {
@@ -684,7 +686,8 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm) {
+decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
+              const __grid_constant__ CUtensorMap tm_pair) {
     extern __shared__ uint8_t smem_raw[];
     Shared sh;
     {
@@ -715,7 +718,8 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm) {
         ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + 0), kPReadyTx);
         ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + 1), kPReadyTx);
         ptx::mbar_arrive_expect_tx(sh.bar(kBarQReady), kQReadyTx);
-        ptx::prefetch_tensormap(&tm);
+        ptx::prefetch_tensormap(&tm_page);
+        ptx::prefetch_tensormap(&tm_pair);
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc_pair(ptx::smem_u32(sh.tmem_slot()), kTmemCols);
@@ -730,7 +734,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm) {
     if (warp < kWarpProducer) {
         run_softmax(p, sh, tmem, crank, warp, lane);
     } else if (warp == kWarpProducer) {
-        if (lane == 0) run_producer(p, sh, &tm, crank);
+        if (lane == 0) run_producer(p, sh, &tm_page, &tm_pair, crank);
     } else if (warp == kWarpMma) {
         if (lane == 0 && crank == 0) run_mma(p, sh, tmem);
     }

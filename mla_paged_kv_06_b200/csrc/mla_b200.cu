@@ -128,6 +128,21 @@ EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
+// 3-D view of the page pool for the split kernel: {64 elements, num_blocks * 64 rows
+// (stride 1152 bytes), 9 chunks of 128 bytes (stride 128 bytes)}, 128-byte swizzle, box
+// {64, 64, box_chunks}: a box lands as box_chunks consecutive 64-row x 128-byte tiles.
+bool make_page_map(CUtensorMap* map, const void* kcache, int num_blocks, int box_chunks) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, (cuuint64_t)num_blocks * kBlock, (cuuint64_t)(kHeadDim / 64)};
+    const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kBlock, (cuuint32_t)box_chunks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kcache), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2D view of the page pool: [num_blocks * 64 rows][576 bf16], row stride 1152 bytes.
 bool make_pool_map(CUtensorMap* map, const void* kcache, int num_blocks, int box_cols,
                    CUtensorMapSwizzle swz) {
@@ -311,10 +326,12 @@ mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blo
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
     const int pairs = device_pairs(dev);
     if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
-    CUtensorMap tm;
-    if (!make_pool_map(&tm, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    CUtensorMap tm_page, tm_pair;
+    if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
+        !make_page_map(&tm_pair, kcache, num_blocks, 2))
+        return MLA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm);
+    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return launch_combine(p, s);
 }
@@ -343,10 +360,12 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
     DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
                                  batch, s_q, h_q, scale, causal, metadata, num_splits,
                                  scratch, scratch_bytes, out, lse);
-    CUtensorMap tm;
-    if (!make_pool_map(&tm, kcache, num_blocks, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    CUtensorMap tm_page, tm_pair;
+    if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
+        !make_page_map(&tm_pair, kcache, num_blocks, 2))
+        return MLA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm);
+    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return launch_combine(p, s);
 }
