@@ -36,7 +36,10 @@
 //             The pool is seen as a 3-D tensor {64 elements, rows, 9 chunks of 128 B}, so
 //             one instruction lands a page as its 9 swizzled tiles (the TMA unit streams
 //             8 KB boxes at barely half the rate of whole pages) and a reload is two
-//             2-tile instructions.
+//             2-tile instructions. It also brings each item's 64 q rows: dims
+//             [256,576) straight into their tiles, dims [0,256) into the (then idle) P
+//             buffers, from where the softmax warps move them into TMEM. So the next
+//             item's QK overlaps the previous item's epilogue.
 //   warp 9    TMEM owner (both CTAs) and, in CTA 0, the MMA issuer.
 // CTA 1's warps tell CTA 0's barriers that their Q or P is ready with a 4-byte
 // asynchronous store whose completion counts bytes on the barrier (release at cluster
@@ -85,8 +88,10 @@ enum : uint32_t {
     kBarVFull = kBarQkDone + 2,     // [2] this CTA's reload landed
     kBarPReady = kBarVFull + 2,     // [2] P written and V ready in both CTAs (CTA 0's used)
     kBarPvDone = kBarPReady + 2,    // [2] PV of the step done (both CTAs)
-    kBarQReady = kBarPvDone + 2,    // Q of the item loaded in both CTAs (CTA 0's used)
-    kBarMaxX = kBarQReady + 1,      // [2 groups] row-max halves posted
+    kBarQReady = kBarPvDone + 2,    // Q of the item in place in both CTAs (CTA 0's used)
+    kBarQLand = kBarQReady + 1,     // the item's q rows landed in shared memory
+    kBarOFree = kBarQLand + 1,      // O of the previous item read out in both CTAs (CTA 0's)
+    kBarMaxX = kBarOFree + 1,       // [2 groups] row-max halves posted
     kBarMref = kBarMaxX + 2,        // [2 groups] reference max of the step posted
     kBarLsum = kBarMref + 2,        // both groups posted their row sums
     kBarDrain = kBarLsum + 1,       // the MMA issuer's last commit
@@ -96,6 +101,8 @@ constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort flag
 // bytes CTA 1 signals per phase: one 4-byte store per softmax warp that arrives
 constexpr uint32_t kPReadyTx = 4 * 4;
 constexpr uint32_t kQReadyTx = 8 * 4;
+constexpr uint32_t kOFreeTx = 8 * 4;
+constexpr uint32_t kQBytes = 9 * kBoxBytes;             // 64 q rows x 576 dims
 constexpr uint32_t kSmemBytes = kOffMisc + 16;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;      // room to align the base to 1 KB
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
@@ -219,11 +226,25 @@ __device__ __forceinline__ int page_row(const DecodeParams& p, int b, int k, int
 // four boxes that only QK needed (CTA 0: boxes 2,3,6,7 <- page B's 0,1,4,5; CTA 1: boxes
 // 0,1,4,5 <- page A's 2,3,6,7), completing on this CTA's own barrier.
 __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared& sh,
-                                             const CUtensorMap* tm_page,
-                                             const CUtensorMap* tm_pair, uint32_t crank) {
+                                             const CUtensorMap* tm_page, const CUtensorMap* tm_pair,
+                                             const CUtensorMap* tm_q4, const CUtensorMap* tm_q5,
+                                             uint32_t crank) {
     ItemIter iter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item it;
     bool have = iter.next(it);
+    // q stream: item m's rows may land once PV of item m-1's last step is done (the q
+    // tiles, Q in TMEM and the P buffers are then free)
+    ItemIter qiter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
+    Item qit;
+    bool qhave = qiter.next(qit);
+    uint32_t qitems = 0;
+    int64_t q_prev_last = -1;                      // global last step of the previous item
+    uint32_t q_first = 0;                          // global first step of item qit
+    auto q_row = [&](const Item& x) { return (x.b * p.rows + x.t * kTileRows) + 64 * (int)crank; };
+    if (qhave) {
+        ptx::tma_prefetch_3d(tm_q5, 0, q_row(qit), 4);
+        ptx::tma_prefetch_3d(tm_q4, 0, q_row(qit), 0);
+    }
     int j = 0;                                     // step within the current item
     ItemIter piter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item pit;
@@ -245,10 +266,32 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
     const uint32_t kfull_leader = ptx::mapa(sh.bar(kBarKFull), 0);
     int reload_row[4];                             // pool row of the other page, per step % 4
     uint32_t gk = 0, gv = 0;                       // steps loaded / reloaded
+    // PV completions are observed strictly in step order: PV of step pv_seen + 2 needs
+    // that step's page, which is only loaded after PV of step pv_seen was seen, so the
+    // phase tested below can never be confused with an older one of the same parity
+    uint32_t pv_seen = 0;
     uint64_t t0 = 0;
     uint32_t idle = 0;
     for (;;) {
-        if (gv < gk && ptx::mbar_test_wait(sh.bar(kBarQkDone + (gv & 1u)), (gv >> 1) & 1u)) {
+        if (pv_seen < gk &&
+            ptx::mbar_test_wait(sh.bar(kBarPvDone + (pv_seen & 1u)), (pv_seen >> 1) & 1u))
+            ++pv_seen;
+        if (qhave && (int64_t)pv_seen > q_prev_last) {
+            const uint32_t land = sh.bar(kBarQLand);
+            ptx::mbar_arrive_expect_tx(land, kQBytes);
+            const int y = q_row(qit);
+            ptx::tma_load_3d(sh.base_u32 + kOffQs, tm_q5, land, 0, y, 4);
+            ptx::tma_load_3d(sh.base_u32 + kOffP, tm_q4, land, 0, y, 0);
+            q_first += (uint32_t)qit.steps();
+            q_prev_last = (int64_t)q_first - 1;
+            ++qitems;
+            qhave = qiter.next(qit);
+            if (qhave) {                           // warm L2 for the next item's rows
+                ptx::tma_prefetch_3d(tm_q5, 0, q_row(qit), 4);
+                ptx::tma_prefetch_3d(tm_q4, 0, q_row(qit), 0);
+            }
+            idle = 0;
+        } else if (gv < gk && ptx::mbar_test_wait(sh.bar(kBarQkDone + (gv & 1u)), (gv >> 1) & 1u)) {
             const uint32_t full = sh.bar(kBarVFull + (gv & 1u));
             ptx::mbar_arrive_expect_tx(full, kReloadBytes);
             const uint32_t st = sh.stage(gv & 1u);
@@ -263,9 +306,7 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             }
             ++gv;
             idle = 0;
-        } else if (have && gk < gv + 2 &&
-                   (gk < 2 || ptx::mbar_test_wait(sh.bar(kBarPvDone + (gk & 1u)),
-                                                  ((gk - 2) >> 1) & 1u))) {
+        } else if (have && gk < gv + 2 && gk < pv_seen + 2) {
             const int ka = it.k_lo + 2 * j;
             const int own = page_row(p, it.b, ka + (int)crank, it.k_hi);
             reload_row[gk & 3u] = page_row(p, it.b, ka + (int)(crank ^ 1u), it.k_hi);
@@ -279,7 +320,7 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
                 j = 0;
             }
             idle = 0;
-        } else if (!have && gv == gk) {
+        } else if (!have && gv == gk && !qhave) {
             break;
         } else if ((++idle & 1023u) == 0) {
             if (*sh.abort_flag()) return;
@@ -292,7 +333,8 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             }
         }
     }
-    // the last reloads must land before this CTA may finish
+    // the last copies must land before this CTA may finish
+    if (qitems > 0) wait_bar<false>(sh, sh.bar(kBarQLand), (qitems - 1) & 1u, 0x12u);
     for (uint32_t i = 0; i < 2 && i < gv; ++i) {
         const uint32_t g = gv - 1 - i;
         wait_bar<false>(sh, sh.bar(kBarVFull + (g & 1u)), (g >> 1) & 1u, 0x11u);
@@ -354,6 +396,7 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Shared& sh,
         if (!wait_bar<true>(sh, sh.bar(kBarQReady), items & 1u, 0x20u)) break;
         ptx::mbar_arrive_expect_tx(sh.bar(kBarQReady), kQReadyTx);      // the next item's
         ptx::tc_fence_after();
+        bool o_free = items == 0;        // the previous item's O must be read out first
         const uint32_t n = (uint32_t)it.steps();
         uint32_t qk = 0, pv = 0;
         uint64_t t0 = 0;
@@ -361,7 +404,13 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Shared& sh,
         bool ok = true;
         while (pv < n) {
             const uint32_t Sv = S0 + pv, Sq = S0 + qk;
-            if (pv < qk &&
+            if (!o_free &&
+                ptx::mbar_test_wait_cluster(sh.bar(kBarOFree), (items - 1) & 1u)) {
+                ptx::mbar_arrive_expect_tx(sh.bar(kBarOFree), kOFreeTx);   // this item's
+                ptx::tc_fence_after();
+                o_free = true;
+            }
+            if (pv < qk && (pv > 0 || o_free) &&
                 ptx::mbar_test_wait_cluster(sh.bar(kBarPReady + (Sv & 1u)), (Sv >> 1) & 1u)) {
                 issue_pv(sh, tmem, Sv, pv == 0);
                 ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + (Sv & 1u)), kPReadyTx);  // step Sv+2
@@ -554,6 +603,92 @@ __device__ __forceinline__ bool softmax_step(const DecodeParams& p, const Shared
     return true;
 }
 
+// Where one item's rows stand once its steps are done: what its epilogue needs.
+struct ItemEnd {
+    Item it;
+    int r, qi;
+    bool row_valid;
+    uint32_t last_step;      // global index of the item's last step
+    RowState st;
+};
+
+// Epilogue of an item for this thread's row: merge the four row sums (two groups x two
+// page halves), then write this lane's 128 output dims (dims block `grp`, half `half`)
+// normalised, with the lse, or the fp32 partial for the combine.
+__device__ __forceinline__ bool epilogue(const DecodeParams& p, const Shared& sh,
+                                         const SoftmaxCtx& c, ItemEnd& e, uint32_t epi_index) {
+    const int row = c.row;
+    const uint32_t Sl = e.last_step;
+    if (!warp_wait_bar<false>(sh, sh.bar(kBarMref + (Sl & 1u)), (Sl >> 1) & 1u, 0x38u)) return false;
+    const float m_fin = *reinterpret_cast<volatile float*>(&sh.fptr(kOffMref)[(Sl & 1u) * 64 + row]);
+    rebase(e.st, m_fin);
+    float* lsum = sh.fptr(kOffLsum);
+    lsum[(c.grp * 2 + c.half) * 64 + row] = e.st.l_sum;
+    ptx::mbar_arrive(sh.bar(kBarLsum));
+    if (!warp_wait_bar<false>(sh, sh.bar(kBarLsum), epi_index & 1u, 0x37u)) return false;
+    if (!warp_wait_bar<false>(sh, sh.bar(kBarPvDone + (Sl & 1u)), (Sl >> 1) & 1u, 0x34u)) return false;
+    ptx::tc_fence_after();
+    volatile float* vl = lsum;
+    const float l_tot = (vl[row] + vl[64 + row]) + (vl[128 + row] + vl[192 + row]);
+    const bool empty = !(l_tot > 0.f);
+    const float inv = empty ? 0.f : 1.f / l_tot;
+    const float lse2 = empty ? -INFINITY : m_fin + __log2f(l_tot);
+    const Item& it = e.it;
+    const bool final_out = it.n_chunks == 1;
+    const bool have_ws = it.part < p.max_chunks;
+    if (!final_out && !have_ws && row == 0 && c.grp == 0 && c.half == 0)
+        record_error(kErrWorkspace, (uint32_t)it.v & 0xffffffu);
+    const int tile_row = (int)c.crank * 64 + row;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+        uint32_t ov[32];
+        ptx::tmem_ld32(c.tmem + c.lane_base + kColO + 128 * c.grp + 32 * cc, ov);
+        if (!e.row_valid) continue;
+        const int col = 256 * c.grp + 128 * c.half + 32 * cc;
+        if (final_out) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)it.b * p.rows + e.r) * kHeadDimV + col);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                uint32_t w[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(f32(ov[8 * k + 2 * h]) * inv,
+                                                              f32(ov[8 * k + 2 * h + 1]) * inv);
+                    w[h] = *reinterpret_cast<uint32_t*>(&b2);
+                }
+                dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        } else if (have_ws) {
+            float4* dst = reinterpret_cast<float4*>(
+                p.ws_o + ((size_t)it.part * kTileRows + tile_row) * kHeadDimV + col);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                dst[k] = make_float4(f32(ov[4 * k]) * inv, f32(ov[4 * k + 1]) * inv,
+                                     f32(ov[4 * k + 2]) * inv, f32(ov[4 * k + 3]) * inv);
+        }
+    }
+    if (e.row_valid && c.grp == 0 && c.half == 0) {
+        if (final_out) {
+            const int h = e.r % p.h_q;
+            p.lse[((size_t)it.b * p.h_q + h) * p.s_q + e.qi] = empty ? -INFINITY : lse2 * kLn2;
+        } else if (have_ws) {
+            p.ws_lse[(size_t)it.part * kTileRows + tile_row] = lse2;
+        }
+    }
+    ptx::tc_fence_before();
+    return true;
+}
+
+// Tell CTA 0's barrier `bar` that this warp is done (local arrive in CTA 0; in CTA 1 a
+// 4-byte store whose completion counts on that barrier).
+__device__ __forceinline__ void signal_leader(const Shared& sh, uint32_t crank, uint32_t bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        if (crank == 0) ptx::mbar_arrive(sh.bar(bar));
+        else ptx::st_async_signal(ptx::mapa(sh.sink(), 0), ptx::mapa(sh.bar(bar), 0));
+    }
+}
+
 __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared& sh, uint32_t tmem,
                                             uint32_t crank, int warp, int lane) {
     SoftmaxCtx c;
@@ -565,52 +700,49 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
     c.half = q >> 1;
     c.grp = warp >> 2;
     const int row = c.row;
+    (void)lane;
 
     ItemIter iter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item it;
     uint32_t S = 0;
     uint32_t items = 0;
+    ItemEnd prev;
+    bool have_prev = false;
     while (iter.next(it)) {
         const int r = it.t * kTileRows + (int)crank * 64 + row;   // query row in the sequence
         const bool row_valid = r < p.rows;
         const int qi = row_valid ? r / p.h_q : 0;
         const int n_vis = row_valid ? visible_tokens(it.L, p.s_q, qi, p.causal) : 0;
 
-        // ---- q of this row: lower 256 latent dims into TMEM (both lane halves hold the
-        // row; group g writes dims [128g, 128g+128)), dims [256, 576) into shared memory
+        // ---- q of this row, dims [0,256): from the P buffers (where the producer landed
+        // them) into TMEM, both lane halves (group g moves dims [128g, 128g+128))
+        if (!warp_wait_bar<false>(sh, sh.bar(kBarQLand), items & 1u, 0x3au)) return;
         {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                p.q + ((size_t)it.b * p.rows + (row_valid ? r : 0)) * kHeadDim);
             const uint32_t qaddr = tmem + c.lane_base + kColQ + 64 * c.grp;
+            const uint32_t stg = sh.base_u32 + kOffP + (uint32_t)row * 128;
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 uint32_t v[32];
+                const uint32_t tile = stg + (uint32_t)(2 * c.grp + cc) * kBoxBytes;
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
-                    uint4 x = row_valid ? __ldg(src + c.grp * 16 + cc * 8 + jj) : make_uint4(0, 0, 0, 0);
-                    v[4 * jj + 0] = x.x; v[4 * jj + 1] = x.y; v[4 * jj + 2] = x.z; v[4 * jj + 3] = x.w;
+                    const uint32_t a = tile + (((uint32_t)jj ^ (uint32_t)(row & 7)) * 16);
+                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(v[4 * jj]), "=r"(v[4 * jj + 1]), "=r"(v[4 * jj + 2]),
+                                   "=r"(v[4 * jj + 3])
+                                 : "r"(a) : "memory");
                 }
                 ptx::tmem_st32(qaddr + 32 * cc, v);
             }
-            // 40 chunks of 16 B per row (dims 256..575) over the 4 (group, half) threads
-            const int part = c.grp * 2 + c.half;
-            const uint32_t qs = sh.base_u32 + kOffQs + (uint32_t)row * 128;
-#pragma unroll
-            for (int e = 0; e < 10; ++e) {
-                const int ch = part * 10 + e;                  // 0..39
-                uint4 x = row_valid ? __ldg(src + 32 + ch) : make_uint4(0, 0, 0, 0);
-                const uint32_t addr = qs + (uint32_t)(ch >> 3) * kBoxBytes +
-                                      (((uint32_t)(ch & 7) ^ (uint32_t)(row & 7)) * 16);
-                ptx::st_shared_v4(addr, x.x, x.y, x.z, x.w);
-            }
-            ptx::fence_proxy_async_smem();
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (crank == 0) ptx::mbar_arrive(sh.bar(kBarQReady));
-                else ptx::st_async_signal(ptx::mapa(sh.sink(), 0), ptx::mapa(sh.bar(kBarQReady), 0));
-            }
+            signal_leader(sh, crank, kBarQReady);
+        }
+
+        // ---- the previous item's epilogue overlaps this item's first QK
+        if (have_prev) {
+            if (!epilogue(p, sh, c, prev, items - 1)) return;
+            signal_leader(sh, crank, kBarOFree);
         }
 
         RowState st{-INFINITY, 0.f};
@@ -622,72 +754,22 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
         }
         if (!ok) return;
         S = S0 + n;
-
-        // ---- epilogue: this lane's half of dims block `grp` (128 output dims)
-        const uint32_t Sl = S - 1;
-        if (!warp_wait_bar<false>(sh, sh.bar(kBarMref + (Sl & 1u)), (Sl >> 1) & 1u, 0x38u)) return;
-        const float m_fin = *reinterpret_cast<volatile float*>(&sh.fptr(kOffMref)[(Sl & 1u) * 64 + row]);
-        rebase(st, m_fin);
-        float* lsum = sh.fptr(kOffLsum);
-        lsum[(c.grp * 2 + c.half) * 64 + row] = st.l_sum;
-        ptx::mbar_arrive(sh.bar(kBarLsum));
-        if (!warp_wait_bar<false>(sh, sh.bar(kBarLsum), items & 1u, 0x37u)) return;
-        if (!warp_wait_bar<false>(sh, sh.bar(kBarPvDone + (Sl & 1u)), (Sl >> 1) & 1u, 0x34u)) return;
-        ptx::tc_fence_after();
-        volatile float* vl = lsum;
-        const float l_tot = (vl[row] + vl[64 + row]) + (vl[128 + row] + vl[192 + row]);
-        const bool empty = !(l_tot > 0.f);
-        const float inv = empty ? 0.f : 1.f / l_tot;
-        const float lse2 = empty ? -INFINITY : m_fin + __log2f(l_tot);
-        const bool final_out = it.n_chunks == 1;
-        const bool have_ws = it.part < p.max_chunks;
-        if (!final_out && !have_ws && row == 0 && c.grp == 0 && c.half == 0)
-            record_error(kErrWorkspace, (uint32_t)it.v & 0xffffffu);
-        const int tile_row = (int)crank * 64 + row;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-            uint32_t ov[32];
-            ptx::tmem_ld32(tmem + c.lane_base + kColO + 128 * c.grp + 32 * cc, ov);
-            if (!row_valid) continue;
-            const int col = 256 * c.grp + 128 * c.half + 32 * cc;
-            if (final_out) {
-                uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)it.b * p.rows + r) * kHeadDimV + col);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(f32(ov[8 * e + 2 * h]) * inv,
-                                                                  f32(ov[8 * e + 2 * h + 1]) * inv);
-                        w[h] = *reinterpret_cast<uint32_t*>(&b2);
-                    }
-                    dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            } else if (have_ws) {
-                float4* dst = reinterpret_cast<float4*>(
-                    p.ws_o + ((size_t)it.part * kTileRows + tile_row) * kHeadDimV + col);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    dst[e] = make_float4(f32(ov[4 * e]) * inv, f32(ov[4 * e + 1]) * inv,
-                                         f32(ov[4 * e + 2]) * inv, f32(ov[4 * e + 3]) * inv);
-            }
-        }
-        if (row_valid && c.grp == 0 && c.half == 0) {
-            if (final_out) {
-                const int h = r % p.h_q;
-                p.lse[((size_t)it.b * p.h_q + h) * p.s_q + qi] = empty ? -INFINITY : lse2 * kLn2;
-            } else if (have_ws) {
-                p.ws_lse[(size_t)it.part * kTileRows + tile_row] = lse2;
-            }
-        }
-        ptx::tc_fence_before();
+        prev.it = it;
+        prev.r = r;
+        prev.qi = qi;
+        prev.row_valid = row_valid;
+        prev.last_step = S - 1;
+        prev.st = st;
+        have_prev = true;
         ++items;
     }
+    if (have_prev) epilogue(p, sh, c, prev, items - 1);
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
-              const __grid_constant__ CUtensorMap tm_pair) {
+              const __grid_constant__ CUtensorMap tm_pair, const __grid_constant__ CUtensorMap tm_q4,
+              const __grid_constant__ CUtensorMap tm_q5) {
     extern __shared__ uint8_t smem_raw[];
     Shared sh;
     {
@@ -710,6 +792,8 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
             ptx::mbar_init(sh.bar(kBarMref + i), 128);
         }
         ptx::mbar_init(sh.bar(kBarQReady), 8 + 1);              // CTA 0's warps + arming
+        ptx::mbar_init(sh.bar(kBarQLand), 1);
+        ptx::mbar_init(sh.bar(kBarOFree), 8 + 1);               // CTA 0's warps + arming
         ptx::mbar_init(sh.bar(kBarLsum), kSoftmaxThreads);
         ptx::mbar_init(sh.bar(kBarDrain), 1);
         *sh.abort_flag() = 0;
@@ -718,8 +802,11 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
         ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + 0), kPReadyTx);
         ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + 1), kPReadyTx);
         ptx::mbar_arrive_expect_tx(sh.bar(kBarQReady), kQReadyTx);
+        ptx::mbar_arrive_expect_tx(sh.bar(kBarOFree), kOFreeTx);
         ptx::prefetch_tensormap(&tm_page);
         ptx::prefetch_tensormap(&tm_pair);
+        ptx::prefetch_tensormap(&tm_q4);
+        ptx::prefetch_tensormap(&tm_q5);
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc_pair(ptx::smem_u32(sh.tmem_slot()), kTmemCols);
@@ -734,7 +821,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
     if (warp < kWarpProducer) {
         run_softmax(p, sh, tmem, crank, warp, lane);
     } else if (warp == kWarpProducer) {
-        if (lane == 0) run_producer(p, sh, &tm_page, &tm_pair, crank);
+        if (lane == 0) run_producer(p, sh, &tm_page, &tm_pair, &tm_q4, &tm_q5, crank);
     } else if (warp == kWarpMma) {
         if (lane == 0 && crank == 0) run_mma(p, sh, tmem);
     }

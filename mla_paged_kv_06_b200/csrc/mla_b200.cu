@@ -143,6 +143,19 @@ bool make_page_map(CUtensorMap* map, const void* kcache, int num_blocks, int box
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same 3-D view of q ([total rows][576] bf16): box {64, 64 rows, box_chunks}.
+bool make_q_map(CUtensorMap* map, const void* q, size_t total_rows, int box_chunks) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {64, (cuuint64_t)total_rows, (cuuint64_t)(kHeadDim / 64)};
+    const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, 128};
+    const cuuint32_t box[3] = {64, 64, (cuuint32_t)box_chunks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2D view of the page pool: [num_blocks * 64 rows][576 bf16], row stride 1152 bytes.
 bool make_pool_map(CUtensorMap* map, const void* kcache, int num_blocks, int box_cols,
                    CUtensorMapSwizzle swz) {
@@ -326,12 +339,15 @@ mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blo
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
     const int pairs = device_pairs(dev);
     if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
-    CUtensorMap tm_page, tm_pair;
+    CUtensorMap tm_page, tm_pair, tm_q4, tm_q5;
+    const size_t q_rows = (size_t)batch * s_q * h_q;
     if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
-        !make_page_map(&tm_pair, kcache, num_blocks, 2))
+        !make_page_map(&tm_pair, kcache, num_blocks, 2) ||
+        !make_q_map(&tm_q4, q, q_rows, 4) || !make_q_map(&tm_q5, q, q_rows, 5))
         return MLA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair);
+    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair,
+                                                                          tm_q4, tm_q5);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return launch_combine(p, s);
 }
@@ -360,12 +376,15 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
     DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
                                  batch, s_q, h_q, scale, causal, metadata, num_splits,
                                  scratch, scratch_bytes, out, lse);
-    CUtensorMap tm_page, tm_pair;
+    CUtensorMap tm_page, tm_pair, tm_q4, tm_q5;
+    const size_t q_rows = (size_t)batch * s_q * h_q;
     if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
-        !make_page_map(&tm_pair, kcache, num_blocks, 2))
+        !make_page_map(&tm_pair, kcache, num_blocks, 2) ||
+        !make_q_map(&tm_q4, q, q_rows, 4) || !make_q_map(&tm_q5, q, q_rows, 5))
         return MLA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair);
+    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair,
+                                                                          tm_q4, tm_q5);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return launch_combine(p, s);
 }
