@@ -241,19 +241,18 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
     int64_t q_prev_last = -1;                      // global last step of the previous item
     uint32_t q_first = 0;                          // global first step of item qit
     auto q_row = [&](const Item& x) { return (x.b * p.rows + x.t * kTileRows) + 64 * (int)crank; };
-    if (qhave) {
-        ptx::tma_prefetch_3d(tm_q5, 0, q_row(qit), 4);
-        ptx::tma_prefetch_3d(tm_q4, 0, q_row(qit), 0);
-    }
     int j = 0;                                     // step within the current item
     ItemIter piter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item pit;
     bool phave = piter.next(pit);
     int pj = 0;
-    auto prefetch_next = [&]() {
+    // L2 prefetch cursor over this CTA's pages, kPrefetchSteps steps ahead of the loads.
+    // The first two steps are loaded at once, so the prefetches start only after them:
+    // at launch every SM's first loads then reach HBM before any prefetch traffic.
+    auto prefetch_next = [&](bool issue) {
         if (!phave) return;
         const int k = pit.k_lo + 2 * pj + (int)crank;
-        if (k < pit.k_hi) {
+        if (issue && k < pit.k_hi) {
             const int pid = p.block_table[(size_t)pit.b * p.max_blocks + k];
             if (pid >= 0 && pid < p.num_blocks) ptx::tma_prefetch_3d(tm_page, 0, pid * kBlock, 0);
         }
@@ -262,7 +261,8 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             pj = 0;
         }
     };
-    for (int i = 0; i < kPrefetchSteps; ++i) prefetch_next();
+    prefetch_next(false);
+    prefetch_next(false);
     const uint32_t kfull_leader = ptx::mapa(sh.bar(kBarKFull), 0);
     int reload_row[4];                             // pool row of the other page, per step % 4
     uint32_t gk = 0, gv = 0;                       // steps loaded / reloaded
@@ -313,8 +313,11 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             if (crank == 0) ptx::mbar_arrive_expect_tx(sh.bar(kBarKFull + (gk & 1u)), 2 * kPageBytes);
             const uint32_t st = sh.stage(gk & 1u);
             ptx::tma_load_3d_pair(st, tm_page, kfull_leader + 8 * (gk & 1u), 0, own, 0);
-            prefetch_next();
             ++gk;
+            if (gk == 2)
+                for (int i = 0; i < kPrefetchSteps; ++i) prefetch_next(true);
+            else if (gk > 2)
+                prefetch_next(true);
             if (++j >= it.steps()) {
                 have = iter.next(it);
                 j = 0;
