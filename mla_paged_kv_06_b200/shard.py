@@ -28,7 +28,7 @@ from .workloads import BLOCK_SIZE, DecodeInputs
 
 # Fixed cost of one sequence in pages: the same per-item overhead the split-KV
 # scheduler charges, so a rank of many short sequences is not under-counted.
-SEQUENCE_OVERHEAD_PAGES = 2
+SEQUENCE_OVERHEAD_PAGES = 3
 
 
 def sequence_cost(length: int, tiles: int = 1) -> int:

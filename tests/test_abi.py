@@ -152,7 +152,7 @@ def test_schedule_random_and_balanced():
         meta, ns = mla.mla_plan_host(lens, h_q, s_q, U)
         seen, nblk = _walk(meta, ns, lens, h_q, s_q)
         W = int(meta[5])
-        total = sum(2 + n for n in nblk)
+        total = sum(3 + n for n in nblk)          # 3 pages of fixed cost per work sequence
         assert W == max(-(-total // U), 4)
         # no unit owns more than W pages: the largest unit is within one overhead of ideal
         per_unit = [0] * U
