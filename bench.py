@@ -369,7 +369,7 @@ def main():
 
 
 # Bumped whenever the split kernel changes, so stale ncu traffic is never reported.
-KERNEL_REV = "pair-1"
+KERNEL_REV = "pair-2"
 
 if __name__ == "__main__":
     sys.exit(main())

@@ -53,22 +53,45 @@ combine_kernel(const DecodeParams p) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float lse2 = mx + __log2f(sum);
-    // out = sum_c 2^(lse_c - lse) O_c; lane owns dims [4 lane, 4 lane + 4) and +128 j
+    // out = sum_c 2^(lse_c - lse) O_c; lane owns dims [4 lane, 4 lane + 4) and +128 j.
+    // Chunks go two at a time so both chunks' loads are in flight together (most split
+    // rows have exactly two chunks).
     float acc[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-    for (int c = 0; c < n_chunks; ++c) {
-        const size_t slot = (size_t)(base + c) * kTileRows + r_local;
-        const float w = exp2f(p.ws_lse[slot] - lse2);
-        const float4* src = reinterpret_cast<const float4*>(p.ws_o + slot * kHeadDimV);
+    auto add = [&](const float4 (&x)[4], float w) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const float4 x = src[lane + 32 * j];
-            acc[4 * j + 0] = fmaf(w, x.x, acc[4 * j + 0]);
-            acc[4 * j + 1] = fmaf(w, x.y, acc[4 * j + 1]);
-            acc[4 * j + 2] = fmaf(w, x.z, acc[4 * j + 2]);
-            acc[4 * j + 3] = fmaf(w, x.w, acc[4 * j + 3]);
+            acc[4 * j + 0] = fmaf(w, x[j].x, acc[4 * j + 0]);
+            acc[4 * j + 1] = fmaf(w, x[j].y, acc[4 * j + 1]);
+            acc[4 * j + 2] = fmaf(w, x[j].z, acc[4 * j + 2]);
+            acc[4 * j + 3] = fmaf(w, x[j].w, acc[4 * j + 3]);
         }
+    };
+    int c = 0;
+    for (; c + 2 <= n_chunks; c += 2) {
+        const size_t s0 = (size_t)(base + c) * kTileRows + r_local;
+        const size_t s1 = s0 + kTileRows;
+        const float4* src0 = reinterpret_cast<const float4*>(p.ws_o + s0 * kHeadDimV);
+        const float4* src1 = reinterpret_cast<const float4*>(p.ws_o + s1 * kHeadDimV);
+        float4 x0[4], x1[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            x0[j] = src0[lane + 32 * j];
+            x1[j] = src1[lane + 32 * j];
+        }
+        const float w0 = exp2f(p.ws_lse[s0] - lse2);
+        const float w1 = exp2f(p.ws_lse[s1] - lse2);
+        add(x0, w0);
+        add(x1, w1);
+    }
+    if (c < n_chunks) {
+        const size_t s0 = (size_t)(base + c) * kTileRows + r_local;
+        const float4* src0 = reinterpret_cast<const float4*>(p.ws_o + s0 * kHeadDimV);
+        float4 x0[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x0[j] = src0[lane + 32 * j];
+        add(x0, exp2f(p.ws_lse[s0] - lse2));
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
