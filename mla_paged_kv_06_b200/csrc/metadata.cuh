@@ -7,6 +7,9 @@
 namespace mla {
 
 constexpr int kMetaThreads = 1024;
+// Largest table (cumulative costs C[V+1] and page counts per sequence, int32) the
+// scheduler keeps in shared memory; larger batches use the num_splits buffer itself.
+constexpr size_t kMetaSmemMax = 160 * 1024;
 
 // Block-wide exclusive scan of one int64 per thread; returns the block total.
 __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* smem_warp,
@@ -42,15 +45,29 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* smem
 // {v_begin, page_begin, v_end, page_end, chunk_begin, 0, 0, 0} per unit.
 // num_splits holds the cumulative costs C[v] while the units are located, then is
 // overwritten with the chunk prefix.
+// `in_smem`: the cost table and page counts live in dynamic shared memory (the launch
+// provides (V + 1 + batch) int32), so the per-unit binary searches never wait on L2;
+// otherwise the costs are kept in num_splits and the lengths re-read from seqlens.
 __global__ void __launch_bounds__(kMetaThreads)
 metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q, int tiles,
-                int num_units,
+                int num_units, int in_smem,
                 int32_t* __restrict__ metadata, int32_t* __restrict__ num_splits) {
     __shared__ int64_t warp_sums[33];
     __shared__ int64_t s_total;
+    extern __shared__ int32_t dyn[];
     const int V = batch * tiles;
+    int32_t* Cs = in_smem ? dyn : num_splits;               // cumulative costs C[0..V]
+    int32_t* Ps = in_smem ? dyn + V + 1 : nullptr;          // pages per sequence
+    if (in_smem) {
+        for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+            const int L = seqlens[b];
+            Ps[b] = pages_of(L < 0 ? 0 : L);
+        }
+        __syncthreads();
+    }
     auto pages = [&](int v) {
-        int L = seqlens[v % batch];
+        if (Ps) return (int)Ps[v % batch];
+        const int L = seqlens[v % batch];
         return pages_of(L < 0 ? 0 : L);
     };
 
@@ -64,19 +81,19 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
         int64_t c = carry + pre;
         if (v < V) {
             if (c > 0x7fffffffLL) record_error(kErrBadInput, 0xfffffeu);
-            num_splits[v] = (int32_t)(c > 0x7fffffffLL ? 0x7fffffff : c);
+            Cs[v] = (int32_t)(c > 0x7fffffffLL ? 0x7fffffff : c);
         }
         carry += tot;
     }
     if (threadIdx.x == 0) {
         if (carry > 0x7fffffffLL) { record_error(kErrBadInput, 0xfffffeu); carry = 0x7fffffff; }
-        num_splits[V] = (int32_t)carry;
+        Cs[V] = (int32_t)carry;
         s_total = carry;
     }
     __syncthreads();
     const int64_t total = s_total;
     const int64_t W = unit_cost(total, num_units);
-    auto C = [&](int v) { return (int64_t)num_splits[v]; };
+    auto C = [&](int v) { return (int64_t)Cs[v]; };
 
     // Phase 2: one thread per unit locates its first and one-past-last page.
     for (int u = threadIdx.x; u < num_units; u += blockDim.x) {
@@ -98,7 +115,8 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
     }
     __syncthreads();
 
-    // Phase 3: chunk counts -> exclusive prefix, written over the costs tile by tile.
+    // Phase 3: chunk counts -> exclusive prefix into num_splits (over the costs, tile by
+    // tile, when they were kept there).
     carry = 0;
     for (int base = 0; base < V; base += blockDim.x) {
         int v = base + threadIdx.x;

@@ -70,6 +70,22 @@ bool prepare_split_kernel(int dev) {
     return true;
 }
 
+// Allow the scheduler kernel kMetaSmemMax of dynamic shared memory (once per device).
+bool prepare_metadata_kernel() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    static std::mutex mu;
+    static std::vector<char> done;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)done.size() <= dev) done.resize(dev + 1, 0);
+    if (done[dev]) return done[dev] > 0;
+    const bool ok = cudaFuncSetAttribute(metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kMetaSmemMax) == cudaSuccess;
+    if (!ok) cudaGetLastError();
+    done[dev] = ok ? 1 : -1;
+    return ok;
+}
+
 // 2-CTA clusters of the split kernel that can be co-resident on a device (cached per
 // device); a schedule never uses more units than this, so every unit runs in one wave.
 int device_pairs(int dev) {
@@ -294,8 +310,11 @@ mla_status mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q,
     if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
     const int units = mla_num_work_units(num_sms);
     if (units < 0) return units;
-    metadata_kernel<<<1, kMetaThreads, 0, (cudaStream_t)stream>>>(
-        seqlens, batch, h_q, s_q, num_tiles(h_q, s_q), units, metadata, num_splits);
+    const int tiles = num_tiles(h_q, s_q);
+    const size_t table = ((size_t)batch * tiles + 1 + (size_t)batch) * sizeof(int32_t);
+    const bool in_smem = table <= kMetaSmemMax && prepare_metadata_kernel();
+    metadata_kernel<<<1, kMetaThreads, in_smem ? table : 0, (cudaStream_t)stream>>>(
+        seqlens, batch, h_q, s_q, tiles, units, in_smem ? 1 : 0, metadata, num_splits);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
