@@ -277,37 +277,67 @@ def main():
     if st != 0:
         raise RuntimeError(f"device error during timing: {mla.status_string(st)} {word:#x}")
 
-    # end to end through the public call with host buffers: q, block table and lengths
-    # copied in from pinned memory and out + lse read back every step
+    # End to end through the public calls with host buffers, run the way a serving loop
+    # runs them: every step copies its q, block table and lengths in from pinned host
+    # memory and reads its out and lse back, on their own streams, so that step k+1's
+    # copy-in and step k-1's copy-out overlap step k's compute. Events order every reuse
+    # of the two buffer sets. The KV cache (the step's dominant input) stays resident
+    # as decode state and exceeds L2, so no flush separates these steps.
     hq = x.q.pin_memory()
     hbt = x.block_table.pin_memory()
     hsl = x.seqlens.pin_memory()
-    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    dq = [d["q"], torch.empty_like(d["q"])]
+    dbt = [d["block_table"], torch.empty_like(d["block_table"])]
+    dsl = [d["seqlens"], torch.empty_like(d["seqlens"])]
+    douts = [out, torch.empty_like(out)]
+    dlses = [lse, torch.empty_like(lse)]
+    hout = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+    hlse = [torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True) for _ in range(2)]
     h2d = hq.numel() * 2 + hbt.numel() * 4 + hsl.numel() * 4
-    d2h = hout.numel() * 2 + hlse.numel() * 4
+    d2h = hout[0].numel() * 2 + hlse[0].numel() * 4
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
-    def e2e_step():
-        d["q"].copy_(hq, non_blocking=True)
-        d["block_table"].copy_(hbt, non_blocking=True)
-        d["seqlens"].copy_(hsl, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
+    def run_e2e(n):
+        ev_comp, ev_out = [], []
+        first = torch.cuda.Event(enable_timing=True)
+        first.record(s_in)
+        for k in range(n):
+            i = k % 2
+            if k >= 2:
+                s_in.wait_event(ev_comp[k - 2])          # step k-2 no longer reads set i
+            with torch.cuda.stream(s_in):
+                dq[i].copy_(hq, non_blocking=True)
+                dbt[i].copy_(hbt, non_blocking=True)
+                dsl[i].copy_(hsl, non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(s_in)
+            s_comp.wait_event(ev_in)
+            if k >= 2:
+                s_comp.wait_event(ev_out[k - 2])         # set i's outputs were read back
+            mla.mla_get_metadata(dsl[i], x.h_q, x.s_q, nsm, meta, ns, stream=s_comp)
+            mla.mla_decode_fwd(dq[i], d["kcache"], dbt[i], dsl[i], x.scale, x.causal, meta, ns,
+                               ws, douts[i], dlses[i], stream=s_comp)
+            ec = torch.cuda.Event()
+            ec.record(s_comp)
+            ev_comp.append(ec)
+            s_out.wait_event(ec)
+            with torch.cuda.stream(s_out):
+                hout[i].copy_(douts[i], non_blocking=True)
+                hlse[i].copy_(dlses[i], non_blocking=True)
+            eo = torch.cuda.Event(enable_timing=True)
+            eo.record(s_out)
+            ev_out.append(eo)
+        return first, ev_out[-1]
 
-    for _ in range(3):
-        e2e_step()
     torch.cuda.synchronize()
-    e2e_ms = 0.0
-    for k in range(args.steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        e2e_step()
-        b.record(stream)
-        b.synchronize()
-        e2e_ms += a.elapsed_time(b)
-    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
+    run_e2e(3)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a, b = run_e2e(args.steps)
+    b.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b), dist, "cuda")
+    torch.cuda.synchronize()
 
     hbm_peak, tf_peak, peak_kind = peaks()
     avg_decode_s = statistics.mean(decode_ms) / 1e3
@@ -354,8 +384,12 @@ def main():
             "roofline": roof,
             "e2e": {"value": nbytes * args.steps * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / args.steps,
                     "note": "KV cache resident in HBM as decode state; per-step inputs are "
-                            "q, block table and lengths"},
+                            "q, block table and lengths, copied in from pinned memory, and "
+                            "out + lse read back, every step; copy-in, compute and "
+                            "copy-out of consecutive steps overlap on three streams; the "
+                            "KV cache exceeds L2 (no flush between these steps)"},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
