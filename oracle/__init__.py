@@ -1,4 +1,5 @@
-"""CPU oracle for paged MLA decode (test infrastructure; see mla_decode.py)."""
+"""CPU oracle for paged MLA decode and the cache append (test infrastructure; see
+mla_decode.py and kv_append.py)."""
 
 from .mla_decode import (  # noqa: F401
     combine,
@@ -8,3 +9,4 @@ from .mla_decode import (  # noqa: F401
     gather_tokens,
     visible_tokens,
 )
+from . import kv_append  # noqa: F401,E402
