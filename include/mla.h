@@ -184,6 +184,31 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
                                   uint16_t* out, float* lse, void* stream);
 
 /*
+ * Cache append: writes s_new new latent rows per sequence into the paged cache, the
+ * step that block-based paging implies before each decode (the paging of
+ * «DeepSeek booste les performances des GPU NVIDIA Hopper H800…», tomshardware.fr,
+ * paragraph on block-based paging that allocates memory dynamically; 64-token blocks
+ * per the FlashMLA release article). For each sequence b and j < s_new:
+ *     t = seqlens[b] + j
+ *     kcache[block_table[b][t / 64]][t % 64][0][:] = kv_new[b][j][:]     (576 bf16)
+ * a byte copy; nothing else in the cache changes.
+ *
+ *   kv_new       device bf16 [batch][s_new][576], 16-byte aligned
+ *   block_table  device int32 [batch][max_blocks]: the pages, including the ones the
+ *                new positions fall in (the caller allocates them first)
+ *   seqlens      device int32 [batch]: tokens already cached (not modified: the caller
+ *                advances each length by s_new afterwards)
+ *   kcache       device bf16 [num_blocks][64][1][576], 16-byte aligned, written
+ * Supported: 1 <= s_new <= 16, 1 <= batch <= 65536. Invalid arguments return an error
+ * before any launch. A position past the block table or a block id outside the pool is
+ * a device-side bad input (see mla_get_last_device_error); that row is not written.
+ * Asynchronous on `stream`; allocates nothing.
+ */
+mla_status mla_kv_append(const uint16_t* kv_new, int s_new, const int32_t* block_table,
+                         int max_blocks, const int32_t* seqlens, int batch, uint16_t* kcache,
+                         int num_blocks, void* stream);
+
+/*
  * Reads and clears the device-side error word of the current device after
  * synchronising `stream`. Returns MLA_OK, MLA_ERR_DEVICE_TIMEOUT,
  * MLA_ERR_DEVICE_BAD_INPUT or MLA_ERR_CUDA. *detail (may be NULL) receives the raw

@@ -11,6 +11,7 @@
 
 #include "mla.h"
 
+#include "append.cuh"
 #include "combine.cuh"
 #include "common.cuh"
 #include "decode_simt.cuh"
@@ -406,6 +407,23 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
                                                                           tm_q4, tm_q5);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return launch_combine(p, s);
+}
+
+mla_status mla_kv_append(const uint16_t* kv_new, int s_new, const int32_t* block_table,
+                         int max_blocks, const int32_t* seqlens, int batch, uint16_t* kcache,
+                         int num_blocks, void* stream) {
+    if (!kv_new || !block_table || !seqlens || !kcache) return MLA_ERR_INVALID_ARG;
+    if (num_blocks < 1 || max_blocks < 1 || s_new < 1) return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)kv_new | (uintptr_t)kcache) & 15u) return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)block_table | (uintptr_t)seqlens) & 3u) return MLA_ERR_INVALID_ARG;
+    if (batch < 1 || batch > MLA_MAX_BATCH || s_new > MLA_MAX_S_Q) return MLA_ERR_UNSUPPORTED;
+    const long long rows = (long long)batch * s_new;
+    const int per_cta = kAppendThreads / 32;
+    const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
+    kv_append_kernel<<<grid, kAppendThreads, 0, (cudaStream_t)stream>>>(
+        reinterpret_cast<const uint4*>(kv_new), s_new, block_table, max_blocks, seqlens, batch,
+        reinterpret_cast<uint4*>(kcache), num_blocks);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 mla_status mla_get_last_device_error(void* stream, uint32_t* detail) {

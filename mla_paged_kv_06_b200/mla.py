@@ -53,6 +53,7 @@ def _load() -> ctypes.CDLL:
                                       vp, vp, vp, sz, vp, vp, vp]),
         "mla_decode_fwd_noalloc": (i32, [vp, vp, i32, vp, i32, vp, i32, i32, i32, f32, i32,
                                          vp, vp, vp, vp, vp]),
+        "mla_kv_append": (i32, [vp, i32, vp, i32, vp, i32, vp, i32, vp]),
         "mla_get_last_device_error": (i32, [vp, ctypes.POINTER(ctypes.c_uint32)]),
         "mla_plan_host": (i32, [vp, i32, i32, i32, i32, vp, vp]),
     }
@@ -196,6 +197,20 @@ def mla_decode_fwd_noalloc(q, kcache, block_table, seqlens, scale, causal, metad
         _ptr(seqlens), batch, s_q, h_q, float(scale), int(bool(causal)), _ptr(metadata),
         _ptr(num_splits), _ptr(out), _ptr(lse), _stream(stream)), "mla_decode_fwd_noalloc")
     return out, lse
+
+
+def mla_kv_append(kv_new, block_table, seqlens, kcache, stream=None):
+    """Write kv_new (bf16 [batch, s_new, 576]) at positions seqlens[b] + j of each
+    sequence's pages in kcache (in place). The lengths are not advanced."""
+    assert kv_new.is_cuda and kv_new.dtype == torch.bfloat16 and kv_new.dim() == 3
+    assert kv_new.is_contiguous() and kcache.is_contiguous() and kcache.dtype == torch.bfloat16
+    assert block_table.dtype == torch.int32 and block_table.is_contiguous()
+    assert seqlens.dtype == torch.int32 and seqlens.is_contiguous()
+    batch, s_new, _ = kv_new.shape
+    _check(_lib.mla_kv_append(_ptr(kv_new), s_new, _ptr(block_table), block_table.shape[1],
+                              _ptr(seqlens), batch, _ptr(kcache), kcache.shape[0],
+                              _stream(stream)), "mla_kv_append")
+    return kcache
 
 
 def mla_get_last_device_error(stream=None):

@@ -165,3 +165,18 @@ def test_schedule_random_and_balanced():
 def test_schedule_no_split_with_one_unit():
     meta, ns = mla.mla_plan_host([8192, 3, 65536], 128, 2, 1)
     assert np.all(np.diff(ns) == 1)
+
+
+def test_kv_append_rejects_bad_arguments_before_launch():
+    lib = mla.library()
+    buf = (ctypes.c_uint16 * 2048)()
+    ints = (ctypes.c_int32 * 64)()
+    a = ctypes.addressof(buf)
+    i = ctypes.addressof(ints)
+    # null pointers, bad sizes and misaligned rows fail on the host, before any launch
+    assert lib.mla_kv_append(None, 1, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append(a, 0, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append(a, 1, i, 0, i, 2, a, 8, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append(a + 2, 1, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append(a, 17, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_UNSUPPORTED
+    assert lib.mla_kv_append(a, 1, i, 4, i, 0, a, 8, None) == mla.MLA_ERR_UNSUPPORTED
