@@ -35,6 +35,7 @@ from mla_paged_kv_06_b200 import workloads as wl  # noqa: E402
 from mla_paged_kv_06_b200.shard import max_over_ranks, rank_seed  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
+kBlockRoom = 64                     # tokens per page
 LAUNCHES_PER_STEP = 3               # metadata, split kernel, combine kernel
 
 
@@ -339,6 +340,34 @@ def main():
     e2e_ms = max_over_ranks(a.elapsed_time(b), dist, "cuda")
     torch.cuda.synchronize()
 
+    # Cache append (the step before each decode): one new latent row per sequence of the
+    # batch, into a pool of its own whose last page has room for it.
+    ap = wl.make_paged_inputs([kBlockRoom - 1] * x.batch, 1, 8, seed=args.seed + 7)
+    ap_kc, ap_bt = ap.kcache.cuda(), ap.block_table.cuda()
+    ap_sl = torch.full((x.batch,), kBlockRoom - 1, dtype=torch.int32, device="cuda")
+    ap_new = torch.randn((x.batch, 1, 576), generator=torch.Generator().manual_seed(3)).to(
+        torch.bfloat16).cuda()
+    for _ in range(3):
+        mla.mla_kv_append(ap_new, ap_bt, ap_sl, ap_kc)
+    torch.cuda.synchronize()
+    # replayed from a CUDA graph so the figure is the GPU's, not Python's launch cost
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(args.steps):
+            mla.mla_kv_append(ap_new, ap_bt, ap_sl, ap_kc)
+    graph.replay()
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    graph.replay()
+    eb.record(stream)
+    eb.synchronize()
+    append_us = ea.elapsed_time(eb) * 1e3 / args.steps
+    del graph
+    st, word = mla.mla_get_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the cache append: {mla.status_string(st)} {word:#x}")
+
     hbm_peak, tf_peak, peak_kind = peaks()
     avg_decode_s = statistics.mean(decode_ms) / 1e3
     achieved_gbs = nbytes / avg_decode_s / 1e9
@@ -391,6 +420,11 @@ def main():
                             "copy-out of consecutive steps overlap on three streams; the "
                             "KV cache exceeds L2 (no flush between these steps)"},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "kv_append": {"us_per_call": append_us, "rows": x.batch,
+                          "GB/s": 2 * 1152 * x.batch / (append_us * 1e-6) / 1e9,
+                          "note": "mla_kv_append, one new token per sequence; calls replayed "
+                                  "back to back from a CUDA graph on L2-resident rows (a "
+                                  "latency figure)"},
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x, args.cpu_seconds)

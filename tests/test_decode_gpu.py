@@ -85,6 +85,8 @@ SMALL = [
     ([129, 5], 1, 1, False),
     ([258, 3, 1, 0, 64], 3, 7, True),
     ([2500], 1, 100, False),
+    ([300, 70], 16, 64, True),        # the largest row count: 1024 rows, 8 tiles
+    ([1000], 8, 128, True),
 ]
 
 
