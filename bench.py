@@ -37,6 +37,7 @@ from mla_paged_kv_06_b200.shard import max_over_ranks, rank_seed  # noqa: E402
 L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
 kBlockRoom = 64                     # tokens per page
 LAUNCHES_PER_STEP = 3               # metadata, split kernel, combine kernel
+SPLIT_KV_WORLD = 4                  # ranks of the split-KV-across-devices measurement
 
 
 def parse():
@@ -49,6 +50,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--split-kv", type=int, default=SPLIT_KV_WORLD,
+                    help="ranks of the split-KV-across-devices timing (<= 1 skips it)")
     return ap.parse_args()
 
 
@@ -205,6 +208,76 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------------
+def time_split_kv(mla, x, flush, stream, steps):
+    """Split-KV across devices, its device work timed on this GPU: the batch's pages
+    split over SPLIT_KV_WORLD ranks (splitkv.plan_kv_split), each rank's slice decoded to
+    fp32 partials (mla_get_metadata + mla_decode_fwd_partial, L2 flushed before each
+    call, as in the main measurement) one rank after another, then the merge of the
+    stacked parts (mla_combine_partials). The all-gather between the ranks' GPUs is not
+    part of it: its size is reported instead."""
+    from mla_paged_kv_06_b200 import splitkv
+    world = SPLIT_KV_WORLD
+    plan = splitkv.plan_kv_split(x.seqlens, world, x.s_q, x.causal)
+    nsm = mla.default_num_sms()
+    rank_us, rank_gbs, parts_o, parts_l = [], [], [], []
+    for g in range(world):
+        xr = splitkv.make_kv_slice(x, plan, g)
+        q, kc, bt, sl = xr.q.cuda(), xr.kcache.cuda(), xr.block_table.cuda(), xr.seqlens.cuda()
+        meta = torch.empty(mla.mla_metadata_ints(nsm), dtype=torch.int32, device="cuda")
+        ns = torch.empty(mla.mla_num_splits_len(xr.batch, xr.h_q, xr.s_q), dtype=torch.int32,
+                         device="cuda")
+        ws = torch.empty(mla.mla_workspace_bytes(xr.batch, xr.h_q, xr.s_q, nsm),
+                         dtype=torch.uint8, device="cuda")
+        o = torch.empty((xr.batch, xr.s_q, xr.h_q, 512), dtype=torch.float32, device="cuda")
+        lse = torch.empty((xr.batch, xr.h_q, xr.s_q), dtype=torch.float32, device="cuda")
+
+        def call():
+            mla.mla_get_metadata(sl, xr.h_q, xr.s_q, nsm, meta, ns)
+            mla.mla_decode_fwd_partial(q, kc, bt, sl, xr.scale, xr.causal, meta, ns, ws, o, lse)
+
+        for _ in range(3):
+            flush.zero_()
+            call()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        us = statistics.median(ts)
+        nb, _ = wl.algorithmic_work(xr.seqlens, xr.s_q, xr.h_q, xr.causal)
+        rank_us.append(us)
+        rank_gbs.append(nb / (us * 1e-6) / 1e9)
+        parts_o.append(o)
+        parts_l.append(lse)
+        del q, kc, bt, sl, ws
+    o_parts, l_parts = torch.stack(parts_o), torch.stack(parts_l)
+    out = torch.empty((x.batch, x.s_q, x.h_q, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        mla.mla_combine_partials(o_parts, l_parts, out, lse)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        mla.mla_combine_partials(o_parts, l_parts, out, lse)
+    b.record(stream)
+    b.synchronize()
+    combine_us = a.elapsed_time(b) * 1e3 / steps
+    st, word = mla.mla_get_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the split-KV timing: {mla.status_string(st)} {word:#x}")
+    exchange = x.batch * x.s_q * x.h_q * (512 + 1) * 4
+    return {"world": world, "rank_decode_us": rank_us, "rank_GB/s": rank_gbs,
+            "combine_us": combine_us, "exchange_bytes_per_rank": exchange,
+            "note": f"each rank holds about 1/{world} of every sequence's pages; rank decodes "
+                    "(fp32 partials, L2 flushed before each) and the merge of the gathered "
+                    "parts timed one after another on this GPU; the all-gather of "
+                    "exchange_bytes_per_rank per rank between GPUs is not timed"}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -368,6 +441,8 @@ def main():
     if st != 0:
         raise RuntimeError(f"device error in the cache append: {mla.status_string(st)} {word:#x}")
 
+    split_kv = time_split_kv(mla, x, flush, stream, args.steps) if args.split_kv > 1 else None
+
     hbm_peak, tf_peak, peak_kind = peaks()
     avg_decode_s = statistics.mean(decode_ms) / 1e3
     achieved_gbs = nbytes / avg_decode_s / 1e9
@@ -425,6 +500,7 @@ def main():
                           "note": "mla_kv_append, one new token per sequence; calls replayed "
                                   "back to back from a CUDA graph on L2-resident rows (a "
                                   "latency figure)"},
+            "split_kv": split_kv,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x, args.cpu_seconds)
@@ -437,7 +513,7 @@ def main():
 
 
 # Bumped whenever the split kernel changes, so stale ncu traffic is never reported.
-KERNEL_REV = "pair-2"
+KERNEL_REV = "pair-3"
 
 if __name__ == "__main__":
     sys.exit(main())

@@ -79,6 +79,7 @@ typedef int mla_status;
 #define MLA_MAX_BATCH     65536
 #define MLA_METADATA_INTS_PER_UNIT 8
 #define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)  /* scratch of mla_decode_fwd_noalloc */
+#define MLA_MAX_PARTS      1024   /* parts mla_combine_partials merges            */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* mla_status_string(mla_status status);
@@ -182,6 +183,48 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
                                   float scale, int causal,
                                   const int32_t* metadata, const int32_t* num_splits,
                                   uint16_t* out, float* lse, void* stream);
+
+/*
+ * mla_decode_fwd with an fp32 output: identical arguments, layouts, checks and
+ * results, except that `out_f32` (device fp32 [batch][s_q][h_q][512], 16-byte aligned)
+ * receives the normalised output unrounded instead of a bf16 `out`. It gives the
+ * per-device partials of a split across devices (mla_combine_partials), where a bf16
+ * rounding of every partial would add up. A row with no visible token gets out = 0,
+ * lse = -inf, as in mla_decode_fwd.
+ */
+mla_status mla_decode_fwd_partial(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                                  const int32_t* block_table, int max_blocks,
+                                  const int32_t* seqlens, int batch, int s_q, int h_q,
+                                  float scale, int causal,
+                                  const int32_t* metadata, const int32_t* num_splits,
+                                  void* workspace, size_t workspace_bytes,
+                                  float* out_f32, float* lse, void* stream);
+
+/*
+ * Split-KV across devices: merges `parts` partial results of the same query rows,
+ * each computed (by mla_decode_fwd_partial, usually on another device) over a disjoint
+ * token range of every sequence. This is the split-KV combine of mla_decode_fwd (the
+ * FlashMLA release article, paragraph on dynamic sequence handling) with the parts
+ * coming from devices instead of work units; the pages describe no multi-device
+ * decode, so the partitioning across devices is this library's addition. For each
+ * row r of sequence b, with lse_g the part's natural-log lse:
+ *     lse = ln sum_g exp(lse_g)
+ *     out = sum_g exp(lse_g - lse) * O_g                  (bf16, round-to-nearest-even)
+ * Parts with lse_g = -inf weigh nothing (their O_g is not read); a row that no part
+ * sees gets out = 0, lse = -inf.
+ *
+ *   o_parts    device fp32 [parts][batch][s_q][h_q][512], 16-byte aligned (read)
+ *   lse_parts  device fp32 [parts][batch][h_q][s_q] (read)
+ *   out        device bf16 [batch][s_q][h_q][512], 16-byte aligned (written)
+ *   lse        device fp32 [batch][h_q][s_q] (written)
+ * Supported: 1 <= parts <= MLA_MAX_PARTS and the shapes of mla_decode_fwd. Invalid
+ * arguments return an error before any launch. Asynchronous on `stream`; allocates
+ * nothing. The caller gathers the parts into one buffer first (an all-gather over the
+ * devices of the split).
+ */
+mla_status mla_combine_partials(const float* o_parts, const float* lse_parts, int parts,
+                                int batch, int s_q, int h_q, uint16_t* out, float* lse,
+                                void* stream);
 
 /*
  * Cache append: writes s_new new latent rows per sequence into the paged cache, the

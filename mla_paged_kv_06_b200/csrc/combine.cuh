@@ -2,7 +2,8 @@
 // normalised output O_c and the log2-domain lse_c of its token subset; the softmax over
 // the union weighs chunk c by 2^(lse_c - lse) with lse = log2 sum_c 2^lse_c. Work
 // sequences that were not split are skipped (the split kernel already wrote them);
-// work sequences that own no page at all (L = 0) get out = 0, lse = -inf here.
+// work sequences that own no page at all (L = 0) get out = 0, lse = -inf here. With
+// p.out_f32 set the merged rows are written there in fp32 instead of to p.out.
 #pragma once
 
 #include "common.cuh"
@@ -11,6 +12,28 @@ namespace mla {
 
 constexpr int kCombineThreads = 256;
 constexpr int kCombineRowsPerCta = kCombineThreads / 32;   // one warp per row
+
+// Row of 512 outputs held as 16 floats per lane: lane owns dims [4 lane + 128 j, +4).
+__device__ __forceinline__ void store_out_row(const DecodeParams& p, size_t row_index,
+                                              const float (&acc)[16], int lane) {
+    if (p.out_f32) {
+        float4* dst = reinterpret_cast<float4*>(p.out_f32 + row_index * kHeadDimV);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            dst[lane + 32 * j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+        return;
+    }
+    uint2* dst = reinterpret_cast<uint2*>(p.out + row_index * kHeadDimV);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[4 * j + 0], acc[4 * j + 1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[4 * j + 2], acc[4 * j + 3]);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        dst[lane + 32 * j] = pk;
+    }
+}
 
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const DecodeParams p) {
@@ -24,13 +47,12 @@ combine_kernel(const DecodeParams p) {
     const int r = t * kTileRows + r_local;
     if (r >= p.rows) return;
     const int i = r / p.h_q, h = r % p.h_q;
-    __nv_bfloat16* dst = p.out + ((size_t)b * p.rows + r) * kHeadDimV;
+    const size_t row_index = (size_t)b * p.rows + r;
+    const float zero[16] = {};
     float* lse_dst = p.lse + ((size_t)b * p.h_q + h) * p.s_q + i;
     if (n_chunks <= 0 || base + n_chunks > p.max_chunks) {
         if (n_chunks > 0 && lane == 0) record_error(kErrWorkspace, (uint32_t)v & 0xffffffu);
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        reinterpret_cast<uint4*>(dst)[lane] = z;
-        reinterpret_cast<uint4*>(dst)[lane + 32] = z;
+        store_out_row(p, row_index, zero, lane);
         if (lane == 0) *lse_dst = -INFINITY;
         return;
     }
@@ -41,9 +63,7 @@ combine_kernel(const DecodeParams p) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (mx == -INFINITY) {   // every chunk empty for this row
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        reinterpret_cast<uint4*>(dst)[lane] = z;
-        reinterpret_cast<uint4*>(dst)[lane + 32] = z;
+        store_out_row(p, row_index, zero, lane);
         if (lane == 0) *lse_dst = -INFINITY;
         return;
     }
@@ -93,15 +113,7 @@ combine_kernel(const DecodeParams p) {
         for (int j = 0; j < 4; ++j) x0[j] = src0[lane + 32 * j];
         add(x0, exp2f(p.ws_lse[s0] - lse2));
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[4 * j + 0], acc[4 * j + 1]);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[4 * j + 2], acc[4 * j + 3]);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi);
-        reinterpret_cast<uint2*>(dst)[lane + 32 * j] = pk;
-    }
+    store_out_row(p, row_index, acc, lane);
     if (lane == 0) *lse_dst = lse2 * kLn2;
 }
 

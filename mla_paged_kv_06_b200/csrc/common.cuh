@@ -30,6 +30,7 @@ struct DecodeParams {
     float* ws_o;                   // [max_chunks][128][512] normalised partial outputs
     __nv_bfloat16* out;            // [batch][s_q][h_q][512]
     float* lse;                    // [batch][h_q][s_q]
+    float* out_f32;                // when set, fp32 [batch][s_q][h_q][512] replaces `out`
     int num_blocks, max_blocks;
     int batch, s_q, h_q, rows, tiles;
     int max_chunks;                // partial slots the workspace holds

@@ -63,7 +63,7 @@ constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
-constexpr int kPrefetchSteps = 3;                    // L2 prefetch distance (steps)
+constexpr int kPrefetchSteps = 1;                    // L2 prefetch distance in steps (fastest of 0-4)
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s per wait, then give up
 
@@ -648,7 +648,14 @@ __device__ __forceinline__ bool epilogue(const DecodeParams& p, const Shared& sh
         ptx::tmem_ld32(c.tmem + c.lane_base + kColO + 128 * c.grp + 32 * cc, ov);
         if (!e.row_valid) continue;
         const int col = 256 * c.grp + 128 * c.half + 32 * cc;
-        if (final_out) {
+        if (final_out && p.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(
+                p.out_f32 + ((size_t)it.b * p.rows + e.r) * kHeadDimV + col);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                dst[k] = make_float4(f32(ov[4 * k]) * inv, f32(ov[4 * k + 1]) * inv,
+                                     f32(ov[4 * k + 2]) * inv, f32(ov[4 * k + 3]) * inv);
+        } else if (final_out) {
             uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)it.b * p.rows + e.r) * kHeadDimV + col);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {

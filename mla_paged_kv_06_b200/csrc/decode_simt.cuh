@@ -28,9 +28,15 @@ __device__ __forceinline__ void simt_store_row(const DecodeParams& p, int b, int
     const float lse2 = empty ? -INFINITY : m2 + __log2f(l);
     if (n_chunks == 1) {
         const int i = r / p.h_q, h = r % p.h_q;
-        __nv_bfloat16* dst = p.out + ((size_t)b * p.rows + r) * kHeadDimV;
+        if (p.out_f32) {
+            float* dst = p.out_f32 + ((size_t)b * p.rows + r) * kHeadDimV;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) dst[lane + 32 * j] = __float2bfloat16_rn(o[j] * inv);
+            for (int j = 0; j < 16; ++j) dst[lane + 32 * j] = o[j] * inv;
+        } else {
+            __nv_bfloat16* dst = p.out + ((size_t)b * p.rows + r) * kHeadDimV;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) dst[lane + 32 * j] = __float2bfloat16_rn(o[j] * inv);
+        }
         if (lane == 0)
             p.lse[((size_t)b * p.h_q + h) * p.s_q + i] = empty ? -INFINITY : lse2 * kLn2;
     } else {

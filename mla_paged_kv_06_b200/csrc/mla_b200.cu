@@ -17,6 +17,7 @@
 #include "decode_simt.cuh"
 #include "decode_pair.cuh"
 #include "metadata.cuh"
+#include "rank_combine.cuh"
 #include "sched.cuh"
 
 // Split-partial scratch of mla_decode_fwd_noalloc: a fixed array inside the library in
@@ -226,6 +227,7 @@ DecodeParams make_params(const uint16_t* q, const uint16_t* kcache, int num_bloc
     p.max_chunks = (int)(cap > 0x7fffffff ? 0x7fffffff : cap);
     p.out = reinterpret_cast<__nv_bfloat16*>(out);
     p.lse = lse;
+    p.out_f32 = nullptr;
     p.num_blocks = num_blocks;
     p.max_blocks = max_blocks;
     p.batch = batch;
@@ -260,6 +262,39 @@ mla_status launch_combine(const DecodeParams& p, cudaStream_t s) {
     dim3 grid(p.batch * p.tiles, kTileRows / kCombineRowsPerCta);
     combine_kernel<<<grid, kCombineThreads, 0, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// mla_decode_fwd and mla_decode_fwd_partial: bf16 `out` or fp32 `out_f32` (one is null).
+mla_status decode_tc(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                     const int32_t* block_table, int max_blocks, const int32_t* seqlens,
+                     int batch, int s_q, int h_q, float scale, int causal,
+                     const int32_t* metadata, const int32_t* num_splits, void* workspace,
+                     size_t workspace_bytes, uint16_t* out, float* out_f32, float* lse,
+                     void* stream) {
+    uint16_t* out_any = out ? out : reinterpret_cast<uint16_t*>(out_f32);
+    mla_status st = validate_decode(q, kcache, num_blocks, block_table, max_blocks, seqlens,
+                                    batch, s_q, h_q, scale, causal, metadata, num_splits,
+                                    workspace, workspace_bytes, out_any, lse);
+    if (st != MLA_OK) return st;
+    DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
+                                 batch, s_q, h_q, scale, causal, metadata, num_splits,
+                                 workspace, workspace_bytes, out, lse);
+    p.out_f32 = out_f32;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    const int pairs = device_pairs(dev);
+    if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
+    CUtensorMap tm_page, tm_pair, tm_q4, tm_q5;
+    const size_t q_rows = (size_t)batch * s_q * h_q;
+    if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
+        !make_page_map(&tm_pair, kcache, num_blocks, 2) ||
+        !make_q_map(&tm_q4, q, q_rows, 4) || !make_q_map(&tm_q5, q, q_rows, 5))
+        return MLA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair,
+                                                                          tm_q4, tm_q5);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    return launch_combine(p, s);
 }
 
 }  // namespace
@@ -348,28 +383,44 @@ mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blo
                           int batch, int s_q, int h_q, float scale, int causal,
                           const int32_t* metadata, const int32_t* num_splits, void* workspace,
                           size_t workspace_bytes, uint16_t* out, float* lse, void* stream) {
-    mla_status st = validate_decode(q, kcache, num_blocks, block_table, max_blocks, seqlens,
-                                    batch, s_q, h_q, scale, causal, metadata, num_splits,
-                                    workspace, workspace_bytes, out, lse);
-    if (st != MLA_OK) return st;
-    DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
-                                 batch, s_q, h_q, scale, causal, metadata, num_splits,
-                                 workspace, workspace_bytes, out, lse);
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-    const int pairs = device_pairs(dev);
-    if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
-    CUtensorMap tm_page, tm_pair, tm_q4, tm_q5;
-    const size_t q_rows = (size_t)batch * s_q * h_q;
-    if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
-        !make_page_map(&tm_pair, kcache, num_blocks, 2) ||
-        !make_q_map(&tm_q4, q, q_rows, 4) || !make_q_map(&tm_q5, q, q_rows, 5))
-        return MLA_ERR_CUDA;
-    cudaStream_t s = (cudaStream_t)stream;
-    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair,
-                                                                          tm_q4, tm_q5);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-    return launch_combine(p, s);
+    return decode_tc(q, kcache, num_blocks, block_table, max_blocks, seqlens, batch, s_q, h_q,
+                     scale, causal, metadata, num_splits, workspace, workspace_bytes, out,
+                     nullptr, lse, stream);
+}
+
+mla_status mla_decode_fwd_partial(const uint16_t* q, const uint16_t* kcache, int num_blocks,
+                                  const int32_t* block_table, int max_blocks,
+                                  const int32_t* seqlens, int batch, int s_q, int h_q,
+                                  float scale, int causal, const int32_t* metadata,
+                                  const int32_t* num_splits, void* workspace,
+                                  size_t workspace_bytes, float* out_f32, float* lse,
+                                  void* stream) {
+    return decode_tc(q, kcache, num_blocks, block_table, max_blocks, seqlens, batch, s_q, h_q,
+                     scale, causal, metadata, num_splits, workspace, workspace_bytes, nullptr,
+                     out_f32, lse, stream);
+}
+
+mla_status mla_combine_partials(const float* o_parts, const float* lse_parts, int parts,
+                                int batch, int s_q, int h_q, uint16_t* out, float* lse,
+                                void* stream) {
+    if (!o_parts || !lse_parts || !out || !lse || parts < 1 || parts > MLA_MAX_PARTS)
+        return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)o_parts | (uintptr_t)out) & 15u) return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)lse_parts | (uintptr_t)lse) & 3u) return MLA_ERR_INVALID_ARG;
+    if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
+    RankCombineParams p;
+    p.o_parts = o_parts;
+    p.lse_parts = lse_parts;
+    p.out = reinterpret_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.parts = parts;
+    p.batch = batch;
+    p.s_q = s_q;
+    p.h_q = h_q;
+    const long long rows = (long long)batch * s_q * h_q;
+    const unsigned grid = (unsigned)((rows + kRankCombineRowsPerCta - 1) / kRankCombineRowsPerCta);
+    rank_combine_kernel<<<grid, kRankCombineThreads, 0, (cudaStream_t)stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int num_blocks,

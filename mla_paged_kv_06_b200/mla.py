@@ -26,6 +26,7 @@ MLA_ERR_WORKSPACE_TOO_SMALL = -4
 MLA_ERR_DEVICE_TIMEOUT = -5
 MLA_ERR_DEVICE_BAD_INPUT = -6
 MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
+MLA_MAX_PARTS = 1024
 
 
 class MlaError(RuntimeError):
@@ -53,6 +54,9 @@ def _load() -> ctypes.CDLL:
                                       vp, vp, vp, sz, vp, vp, vp]),
         "mla_decode_fwd_noalloc": (i32, [vp, vp, i32, vp, i32, vp, i32, i32, i32, f32, i32,
                                          vp, vp, vp, vp, vp]),
+        "mla_decode_fwd_partial": (i32, [vp, vp, i32, vp, i32, vp, i32, i32, i32, f32, i32,
+                                         vp, vp, vp, sz, vp, vp, vp]),
+        "mla_combine_partials": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
         "mla_kv_append": (i32, [vp, i32, vp, i32, vp, i32, vp, i32, vp]),
         "mla_get_last_device_error": (i32, [vp, ctypes.POINTER(ctypes.c_uint32)]),
         "mla_plan_host": (i32, [vp, i32, i32, i32, i32, vp, vp]),
@@ -142,7 +146,8 @@ def mla_get_metadata(seqlens: torch.Tensor, h_q: int, s_q: int, num_sms: int | N
 
 
 def _decode(fn_name, q, kcache, block_table, seqlens, scale, causal, metadata, num_splits,
-            workspace=None, out=None, lse=None, stream=None, num_sms=None):
+            workspace=None, out=None, lse=None, stream=None, num_sms=None,
+            out_dtype=torch.bfloat16):
     assert q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 4 and q.is_contiguous()
     assert kcache.dtype == torch.bfloat16 and kcache.is_contiguous()
     assert block_table.dtype == torch.int32 and block_table.is_contiguous()
@@ -150,7 +155,8 @@ def _decode(fn_name, q, kcache, block_table, seqlens, scale, causal, metadata, n
     num_blocks = kcache.shape[0]
     max_blocks = block_table.shape[1]
     if out is None:
-        out = torch.empty((batch, s_q, h_q, 512), dtype=torch.bfloat16, device=q.device)
+        out = torch.empty((batch, s_q, h_q, 512), dtype=out_dtype, device=q.device)
+    assert out.dtype == out_dtype and out.is_contiguous()
     if lse is None:
         lse = torch.empty((batch, h_q, s_q), dtype=torch.float32, device=q.device)
     if workspace is None:
@@ -171,6 +177,34 @@ def mla_decode_fwd(q, kcache, block_table, seqlens, scale, causal, metadata, num
     lse fp32 [b,h_q,s_q])."""
     return _decode("mla_decode_fwd", q, kcache, block_table, seqlens, scale, causal, metadata,
                    num_splits, workspace, out, lse, stream, num_sms)
+
+
+def mla_decode_fwd_partial(q, kcache, block_table, seqlens, scale, causal, metadata,
+                           num_splits, workspace=None, out=None, lse=None, stream=None,
+                           num_sms=None):
+    """mla_decode_fwd with an unrounded fp32 output (the per-device partial of a split
+    across devices). Returns (out fp32 [b,s_q,h_q,512], lse fp32 [b,h_q,s_q])."""
+    return _decode("mla_decode_fwd_partial", q, kcache, block_table, seqlens, scale, causal,
+                   metadata, num_splits, workspace, out, lse, stream, num_sms,
+                   out_dtype=torch.float32)
+
+
+def mla_combine_partials(o_parts, lse_parts, out=None, lse=None, stream=None):
+    """Merge per-device partials: o_parts fp32 [parts, b, s_q, h_q, 512] and lse_parts
+    fp32 [parts, b, h_q, s_q] -> (out bf16 [b, s_q, h_q, 512], lse fp32 [b, h_q, s_q])."""
+    assert o_parts.is_cuda and o_parts.dtype == torch.float32 and o_parts.dim() == 5
+    assert lse_parts.dtype == torch.float32 and lse_parts.dim() == 4
+    assert o_parts.is_contiguous() and lse_parts.is_contiguous()
+    parts, batch, s_q, h_q, dv = o_parts.shape
+    assert dv == 512 and tuple(lse_parts.shape) == (parts, batch, h_q, s_q)
+    if out is None:
+        out = torch.empty((batch, s_q, h_q, 512), dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((batch, h_q, s_q), dtype=torch.float32, device=o_parts.device)
+    _check(_lib.mla_combine_partials(_ptr(o_parts), _ptr(lse_parts), parts, batch, s_q, h_q,
+                                     _ptr(out), _ptr(lse), _stream(stream)),
+           "mla_combine_partials")
+    return out, lse
 
 
 def mla_decode_fwd_simt(q, kcache, block_table, seqlens, scale, causal, metadata, num_splits,

@@ -180,3 +180,26 @@ def test_kv_append_rejects_bad_arguments_before_launch():
     assert lib.mla_kv_append(a + 2, 1, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_kv_append(a, 17, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_UNSUPPORTED
     assert lib.mla_kv_append(a, 1, i, 4, i, 0, a, 8, None) == mla.MLA_ERR_UNSUPPORTED
+
+
+def test_split_kv_entry_points_reject_bad_arguments_before_launch():
+    lib = mla.library()
+    buf = (ctypes.c_float * 4096)()
+    a = ctypes.addressof(buf)
+    # mla_combine_partials: null pointers, part counts outside [1, MLA_MAX_PARTS],
+    # misaligned buffers and unsupported shapes fail on the host
+    assert lib.mla_combine_partials(None, a, 2, 1, 1, 16, a, a, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_combine_partials(a, a, 0, 1, 1, 16, a, a, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_combine_partials(a, a, mla.MLA_MAX_PARTS + 1, 1, 1, 16, a, a,
+                                    None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_combine_partials(a + 4, a, 2, 1, 1, 16, a, a, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_combine_partials(a, a + 2, 2, 1, 1, 16, a, a, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_combine_partials(a, a, 2, 1, 1, 129, a, a, None) == mla.MLA_ERR_UNSUPPORTED
+    assert lib.mla_combine_partials(a, a, 2, 0, 1, 16, a, a, None) == mla.MLA_ERR_UNSUPPORTED
+    # mla_decode_fwd_partial shares mla_decode_fwd's checks: a null or misaligned fp32
+    # output is refused
+    i = (ctypes.c_int32 * 64)()
+    ip = ctypes.addressof(i)
+    args = lambda out: (a, a, 8, ip, 4, ip, 1, 1, 16, 0.1, 0, ip, ip, a, 1 << 20, out, a, None)
+    assert lib.mla_decode_fwd_partial(*args(None)) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode_fwd_partial(*args(a + 4)) == mla.MLA_ERR_INVALID_ARG
