@@ -513,7 +513,7 @@ def main():
 
 
 # Bumped whenever the split kernel changes, so stale ncu traffic is never reported.
-KERNEL_REV = "pair-3"
+KERNEL_REV = "pair-4"
 
 if __name__ == "__main__":
     sys.exit(main())

@@ -642,40 +642,72 @@ __device__ __forceinline__ bool epilogue(const DecodeParams& p, const Shared& sh
     if (!final_out && !have_ws && row == 0 && c.grp == 0 && c.half == 0)
         record_error(kErrWorkspace, (uint32_t)it.v & 0xffffffu);
     const int tile_row = (int)c.crank * 64 + row;
+    // The rows leave through shared memory, so that each store instruction writes whole
+    // row segments instead of 16 bytes of 32 different rows. A warp stages its 32 rows x
+    // 32 columns in its own 4 KB of the P region: exactly the bytes that only this warp
+    // writes P into (warp 4g + q holds P rows of buffer g, page half q / 2, rows
+    // 32 (q % 2) ..), and every warp moved its q rows out of the region before the row-sum
+    // barrier above. The P buffers are idle here: PV of the item's last step is done and
+    // the next item's first P comes after this epilogue.
+    const int lane = (int)(threadIdx.x & 31);
+    const uint32_t stg = sh.base_u32 + kOffP + (threadIdx.x >> 5) * 4096u;
+    const int row0 = row - lane;                              // the warp's first row
+    const bool fp32_out = !final_out || p.out_f32 != nullptr;
+    float* const f32_base = final_out ? p.out_f32 : p.ws_o;
+    const bool write_any = final_out || have_ws;
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
         uint32_t ov[32];
         ptx::tmem_ld32(c.tmem + c.lane_base + kColO + 128 * c.grp + 32 * cc, ov);
-        if (!e.row_valid) continue;
+        if (!write_any) continue;
         const int col = 256 * c.grp + 128 * c.half + 32 * cc;
-        if (final_out && p.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(
-                p.out_f32 + ((size_t)it.b * p.rows + e.r) * kHeadDimV + col);
+        if (fp32_out) {
+            // stage: lane i's 128-byte row, 16-byte chunks XOR-swizzled by i % 8
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                dst[k] = make_float4(f32(ov[4 * k]) * inv, f32(ov[4 * k + 1]) * inv,
-                                     f32(ov[4 * k + 2]) * inv, f32(ov[4 * k + 3]) * inv);
-        } else if (final_out) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)it.b * p.rows + e.r) * kHeadDimV + col);
+                ptx::st_shared_v4(stg + lane * 128 + ((k ^ (lane & 7)) * 16),
+                                  __float_as_uint(f32(ov[4 * k]) * inv),
+                                  __float_as_uint(f32(ov[4 * k + 1]) * inv),
+                                  __float_as_uint(f32(ov[4 * k + 2]) * inv),
+                                  __float_as_uint(f32(ov[4 * k + 3]) * inv));
+            __syncwarp();
+            // write: 4 rows x 128 bytes per instruction (8 lanes per row)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                uint32_t w[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(f32(ov[8 * k + 2 * h]) * inv,
-                                                              f32(ov[8 * k + 2 * h + 1]) * inv);
-                    w[h] = *reinterpret_cast<uint32_t*>(&b2);
+            for (int i = 0; i < 8; ++i) {
+                const int r = 4 * i + (lane >> 3), k = lane & 7;
+                const uint4 v = ptx::ld_shared_v4(stg + r * 128 + ((k ^ (r & 7)) * 16));
+                const int lr = row0 + r;                          // row within this CTA's 64
+                const int qr = it.t * kTileRows + (int)c.crank * 64 + lr;
+                if (qr < p.rows) {
+                    const size_t grow = final_out ? (size_t)it.b * p.rows + qr
+                                                  : (size_t)it.part * kTileRows + (int)c.crank * 64 + lr;
+                    *reinterpret_cast<uint4*>(f32_base + grow * kHeadDimV + col + 4 * k) = v;
                 }
-                dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
             }
-        } else if (have_ws) {
-            float4* dst = reinterpret_cast<float4*>(
-                p.ws_o + ((size_t)it.part * kTileRows + tile_row) * kHeadDimV + col);
+        } else {
+            // stage: lane i's 64-byte bf16 row, chunks XOR-swizzled by (i / 2) % 4
+            uint32_t w[16];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                dst[k] = make_float4(f32(ov[4 * k]) * inv, f32(ov[4 * k + 1]) * inv,
-                                     f32(ov[4 * k + 2]) * inv, f32(ov[4 * k + 3]) * inv);
+            for (int h = 0; h < 16; ++h) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(f32(ov[2 * h]) * inv, f32(ov[2 * h + 1]) * inv);
+                w[h] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                ptx::st_shared_v4(stg + lane * 64 + ((k ^ ((lane >> 1) & 3)) * 16),
+                                  w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            __syncwarp();
+            // write: 8 rows x 64 bytes per instruction (4 lanes per row)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = 8 * i + (lane >> 2), k = lane & 3;
+                const uint4 v = ptx::ld_shared_v4(stg + r * 64 + ((k ^ ((r >> 1) & 3)) * 16));
+                const int qr = it.t * kTileRows + (int)c.crank * 64 + row0 + r;
+                if (qr < p.rows)
+                    *reinterpret_cast<uint4*>(p.out + ((size_t)it.b * p.rows + qr) * kHeadDimV + col + 8 * k) = v;
+            }
         }
+        __syncwarp();                      // staging reads done before the next chunk's writes
     }
     if (e.row_valid && c.grp == 0 && c.half == 0) {
         if (final_out) {
