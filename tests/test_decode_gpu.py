@@ -116,6 +116,27 @@ def test_device_metadata_matches_host_plan():
             assert np.array_equal(ns.cpu().numpy(), hns)
 
 
+def test_more_units_than_clusters():
+    # A host-planned schedule with more units than the split kernel has clusters: each
+    # cluster then runs several units one after another, and the result is unchanged.
+    mla = _mla()
+    units = 3 * mla.mla_num_work_units(mla.default_num_sms()) + 5
+    lens = [3000, 200, 5000, 64, 1, 0, 777, 4100]
+    x = wl.make_paged_inputs(lens, 1, 128, seed=71, spare_blocks=2, poison=True)
+    hm, hns = mla.mla_plan_host(lens, 128, 1, units)
+    assert int(hm[0]) == units
+    meta = torch.from_numpy(hm).cuda()
+    ns = torch.from_numpy(hns).cuda()
+    d = dict(q=x.q.cuda(), kcache=x.kcache.cuda(), block_table=x.block_table.cuda(),
+             seqlens=x.seqlens.cuda())
+    out, lse = mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
+                                  False, meta, ns, num_sms=2 * units)
+    torch.cuda.synchronize()
+    st, word = mla.mla_get_last_device_error()
+    assert st == mla.MLA_OK, (mla.status_string(st), hex(word))
+    compare(out, lse, *oracle_all(x), what="units > clusters")
+
+
 FULL = ["uniform", "v3", "spec", "skewed"]
 
 
