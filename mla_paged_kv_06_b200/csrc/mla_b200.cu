@@ -349,7 +349,9 @@ mla_status mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q,
     const int tiles = num_tiles(h_q, s_q);
     const size_t table = ((size_t)batch * tiles + 1 + (size_t)batch) * sizeof(int32_t);
     const bool in_smem = table <= kMetaSmemMax && prepare_metadata_kernel();
-    metadata_kernel<<<1, kMetaThreads, in_smem ? table : 0, (cudaStream_t)stream>>>(
+    // a small schedule is latency-bound: fewer threads mean cheaper block-wide scans
+    const int threads = (size_t)batch * tiles <= 8192 ? 256 : kMetaThreads;
+    metadata_kernel<<<1, threads, in_smem ? table : 0, (cudaStream_t)stream>>>(
         seqlens, batch, h_q, s_q, tiles, units, in_smem ? 1 : 0, metadata, num_splits);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
