@@ -1,5 +1,5 @@
-"""CPU oracle for paged MLA decode and the cache append (test infrastructure; see
-mla_decode.py and kv_append.py)."""
+"""CPU oracle for paged MLA decode, the cache append and the FP8 cache format (test
+infrastructure; see mla_decode.py, kv_append.py and fp8_cache.py)."""
 
 from .mla_decode import (  # noqa: F401
     combine,
@@ -9,4 +9,4 @@ from .mla_decode import (  # noqa: F401
     gather_tokens,
     visible_tokens,
 )
-from . import kv_append  # noqa: F401,E402
+from . import fp8_cache, kv_append  # noqa: F401,E402
