@@ -437,6 +437,24 @@ def main():
     eb.synchronize()
     append_us = ea.elapsed_time(eb) * 1e3 / args.steps
     del graph
+    # the same rows quantized into an FP8 cache of the same pages (mla_kv_append_fp8)
+    ap_kc8 = torch.zeros((ap_kc.shape[0], kBlockRoom, mla.MLA_FP8_ROW_BYTES), dtype=torch.uint8,
+                         device="cuda")
+    for _ in range(3):
+        mla.mla_kv_append_fp8(ap_new, ap_bt, ap_sl, ap_kc8)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(args.steps):
+            mla.mla_kv_append_fp8(ap_new, ap_bt, ap_sl, ap_kc8)
+    graph.replay()
+    torch.cuda.synchronize()
+    ea.record(stream)
+    graph.replay()
+    eb.record(stream)
+    eb.synchronize()
+    append_fp8_us = ea.elapsed_time(eb) * 1e3 / args.steps
+    del graph
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the cache append: {mla.status_string(st)} {word:#x}")
@@ -500,6 +518,9 @@ def main():
                           "note": "mla_kv_append, one new token per sequence; calls replayed "
                                   "back to back from a CUDA graph on L2-resident rows (a "
                                   "latency figure)"},
+            "kv_append_fp8": {"us_per_call": append_fp8_us, "rows": x.batch,
+                              "note": "mla_kv_append_fp8: the same rows quantized into the "
+                                      "656-byte FP8 row format, replayed from a CUDA graph"},
             "split_kv": split_kv,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

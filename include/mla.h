@@ -80,6 +80,7 @@ typedef int mla_status;
 #define MLA_METADATA_INTS_PER_UNIT 8
 #define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)  /* scratch of mla_decode_fwd_noalloc */
 #define MLA_MAX_PARTS      1024   /* parts mla_combine_partials merges            */
+#define MLA_FP8_ROW_BYTES   656   /* one token's row in the FP8 cache format        */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* mla_status_string(mla_status status);
@@ -250,6 +251,31 @@ mla_status mla_combine_partials(const float* o_parts, const float* lse_parts, in
 mla_status mla_kv_append(const uint16_t* kv_new, int s_new, const int32_t* block_table,
                          int max_blocks, const int32_t* seqlens, int batch, uint16_t* kcache,
                          int num_blocks, void* stream);
+
+/*
+ * FP8 cache append: quantizes s_new new latent rows per sequence into an FP8 paged cache,
+ * the write side of an FP8 latent cache. The pages fix no FP8 cache format (they use
+ * FP8 for GEMMs with fine-grained scaling factors, the DeepGEMM page on 618zxw.cn); this
+ * one is the library's own. Per token, 656 bytes (MLA_FP8_ROW_BYTES):
+ *     [0, 512)    the 512 latent dims as E4M3 codes (largest finite 448, no infinities)
+ *     [512, 528)  four fp32 scales, one per 128-dim group g: s_g = fp32(amax_g / 448)
+ *     [528, 656)  the 64 rope dims, unchanged bf16
+ * code = E4M3(fp32(x / s_g)), round-to-nearest-even, saturated at +-448; 0 when s_g = 0.
+ * A value reads back as code * s_g. Positions are those of mla_kv_append:
+ *     t = seqlens[b] + j  ->  row t % 64 of page block_table[b][t / 64]
+ *
+ *   kv_new       device bf16 [batch][s_new][576], 16-byte aligned
+ *   block_table, seqlens  as for mla_kv_append (seqlens not modified)
+ *   kcache_fp8   device uint8 [num_blocks][64][656], 16-byte aligned, written
+ * Supported: 1 <= s_new <= 16, 1 <= batch <= 65536. Invalid arguments return an error
+ * before any launch; a position past the block table or a block id outside the pool is a
+ * device-side bad input and that row is not written. A group holding a NaN gets NaN codes
+ * and a NaN scale. Asynchronous on `stream`; allocates nothing. (A decode over this
+ * format is not provided yet.)
+ */
+mla_status mla_kv_append_fp8(const uint16_t* kv_new, int s_new, const int32_t* block_table,
+                             int max_blocks, const int32_t* seqlens, int batch,
+                             uint8_t* kcache_fp8, int num_blocks, void* stream);
 
 /*
  * Reads and clears the device-side error word of the current device after

@@ -12,6 +12,7 @@
 #include "mla.h"
 
 #include "append.cuh"
+#include "append_fp8.cuh"
 #include "combine.cuh"
 #include "common.cuh"
 #include "decode_simt.cuh"
@@ -476,6 +477,23 @@ mla_status mla_kv_append(const uint16_t* kv_new, int s_new, const int32_t* block
     kv_append_kernel<<<grid, kAppendThreads, 0, (cudaStream_t)stream>>>(
         reinterpret_cast<const uint4*>(kv_new), s_new, block_table, max_blocks, seqlens, batch,
         reinterpret_cast<uint4*>(kcache), num_blocks);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status mla_kv_append_fp8(const uint16_t* kv_new, int s_new, const int32_t* block_table,
+                             int max_blocks, const int32_t* seqlens, int batch,
+                             uint8_t* kcache_fp8, int num_blocks, void* stream) {
+    if (!kv_new || !block_table || !seqlens || !kcache_fp8) return MLA_ERR_INVALID_ARG;
+    if (num_blocks < 1 || max_blocks < 1 || s_new < 1) return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)kv_new | (uintptr_t)kcache_fp8) & 15u) return MLA_ERR_INVALID_ARG;
+    if (((uintptr_t)block_table | (uintptr_t)seqlens) & 3u) return MLA_ERR_INVALID_ARG;
+    if (batch < 1 || batch > MLA_MAX_BATCH || s_new > MLA_MAX_S_Q) return MLA_ERR_UNSUPPORTED;
+    const long long rows = (long long)batch * s_new;
+    const int per_cta = kAppendThreads / 32;
+    const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
+    kv_append_fp8_kernel<<<grid, kAppendThreads, 0, (cudaStream_t)stream>>>(
+        reinterpret_cast<const __nv_bfloat16*>(kv_new), s_new, block_table, max_blocks, seqlens,
+        batch, kcache_fp8, num_blocks);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

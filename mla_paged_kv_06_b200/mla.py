@@ -27,6 +27,7 @@ MLA_ERR_DEVICE_TIMEOUT = -5
 MLA_ERR_DEVICE_BAD_INPUT = -6
 MLA_NOALLOC_SCRATCH_BYTES = 64 << 20
 MLA_MAX_PARTS = 1024
+MLA_FP8_ROW_BYTES = 656
 
 
 class MlaError(RuntimeError):
@@ -58,6 +59,7 @@ def _load() -> ctypes.CDLL:
                                          vp, vp, vp, sz, vp, vp, vp]),
         "mla_combine_partials": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
         "mla_kv_append": (i32, [vp, i32, vp, i32, vp, i32, vp, i32, vp]),
+        "mla_kv_append_fp8": (i32, [vp, i32, vp, i32, vp, i32, vp, i32, vp]),
         "mla_get_last_device_error": (i32, [vp, ctypes.POINTER(ctypes.c_uint32)]),
         "mla_plan_host": (i32, [vp, i32, i32, i32, i32, vp, vp]),
     }
@@ -245,6 +247,21 @@ def mla_kv_append(kv_new, block_table, seqlens, kcache, stream=None):
                               _ptr(seqlens), batch, _ptr(kcache), kcache.shape[0],
                               _stream(stream)), "mla_kv_append")
     return kcache
+
+
+def mla_kv_append_fp8(kv_new, block_table, seqlens, kcache_fp8, stream=None):
+    """Quantize kv_new (bf16 [batch, s_new, 576]) into the FP8 cache kcache_fp8 (uint8
+    [num_blocks, 64, 656]) at positions seqlens[b] + j (in place; lengths not advanced)."""
+    assert kv_new.is_cuda and kv_new.dtype == torch.bfloat16 and kv_new.dim() == 3
+    assert kv_new.is_contiguous() and kcache_fp8.is_contiguous()
+    assert kcache_fp8.dtype == torch.uint8 and kcache_fp8.shape[1:] == (64, MLA_FP8_ROW_BYTES)
+    assert block_table.dtype == torch.int32 and block_table.is_contiguous()
+    assert seqlens.dtype == torch.int32 and seqlens.is_contiguous()
+    batch, s_new, _ = kv_new.shape
+    _check(_lib.mla_kv_append_fp8(_ptr(kv_new), s_new, _ptr(block_table), block_table.shape[1],
+                                  _ptr(seqlens), batch, _ptr(kcache_fp8), kcache_fp8.shape[0],
+                                  _stream(stream)), "mla_kv_append_fp8")
+    return kcache_fp8
 
 
 def mla_get_last_device_error(stream=None):

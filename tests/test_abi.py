@@ -203,3 +203,19 @@ def test_split_kv_entry_points_reject_bad_arguments_before_launch():
     args = lambda out: (a, a, 8, ip, 4, ip, 1, 1, 16, 0.1, 0, ip, ip, a, 1 << 20, out, a, None)
     assert lib.mla_decode_fwd_partial(*args(None)) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_decode_fwd_partial(*args(a + 4)) == mla.MLA_ERR_INVALID_ARG
+
+
+def test_kv_append_fp8_rejects_bad_arguments_before_launch():
+    lib = mla.library()
+    buf = (ctypes.c_uint16 * 2048)()
+    ints = (ctypes.c_int32 * 64)()
+    a = ctypes.addressof(buf)
+    i = ctypes.addressof(ints)
+    assert lib.mla_kv_append_fp8(None, 1, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append_fp8(a, 1, i, 4, i, 2, None, 8, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append_fp8(a, 0, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append_fp8(a, 1, i, 4, i, 2, a, 0, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append_fp8(a, 1, i, 4, i, 2, a + 8, 8, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_kv_append_fp8(a, 17, i, 4, i, 2, a, 8, None) == mla.MLA_ERR_UNSUPPORTED
+    assert lib.mla_kv_append_fp8(a, 1, i, 4, i, 0, a, 8, None) == mla.MLA_ERR_UNSUPPORTED
+    assert mla.MLA_FP8_ROW_BYTES == 656
