@@ -38,6 +38,7 @@ L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
 kBlockRoom = 64                     # tokens per page
 LAUNCHES_PER_STEP = 3               # metadata, split kernel, combine kernel
 SPLIT_KV_WORLD = 4                  # ranks of the split-KV-across-devices measurement
+SPLIT_KV_LENGTHS = [65536] * 4      # its sequences: long contexts split over the ranks
 
 
 def parse():
@@ -208,15 +209,17 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------------
-def time_split_kv(mla, x, flush, stream, steps):
-    """Split-KV across devices, its device work timed on this GPU: the batch's pages
-    split over SPLIT_KV_WORLD ranks (splitkv.plan_kv_split), each rank's slice decoded to
-    fp32 partials (mla_get_metadata + mla_decode_fwd_partial, L2 flushed before each
-    call, as in the main measurement) one rank after another, then the merge of the
-    stacked parts (mla_combine_partials). The all-gather between the ranks' GPUs is not
-    part of it: its size is reported instead."""
+def time_split_kv(mla, flush, stream, steps, seed):
+    """Split-KV across devices, its device work timed on this GPU, on the case it is for:
+    a few sequences too long for one GPU's share (SPLIT_KV_LENGTHS tokens, 128 heads).
+    Their pages are split over SPLIT_KV_WORLD ranks (splitkv.plan_kv_split); each rank's
+    slice is decoded to fp32 partials (mla_get_metadata + mla_decode_fwd_partial, L2
+    flushed before each call, as in the main measurement) one rank after another, then
+    the stacked parts are merged (mla_combine_partials). The all-gather between the
+    ranks' GPUs is not part of it: its size is reported instead."""
     from mla_paged_kv_06_b200 import splitkv
     world = SPLIT_KV_WORLD
+    x = wl.make_paged_inputs(SPLIT_KV_LENGTHS, 1, 128, seed=seed + 11)
     plan = splitkv.plan_kv_split(x.seqlens, world, x.s_q, x.causal)
     nsm = mla.default_num_sms()
     rank_us, rank_gbs, parts_o, parts_l = [], [], [], []
@@ -259,23 +262,37 @@ def time_split_kv(mla, x, flush, stream, steps):
     lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
     for _ in range(3):
         mla.mla_combine_partials(o_parts, l_parts, out, lse)
+    torch.cuda.synchronize()
+    # replayed from a CUDA graph: back-to-back calls from Python would time the host
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(steps):
+            mla.mla_combine_partials(o_parts, l_parts, out, lse)
+    graph.replay()
+    torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(steps):
-        mla.mla_combine_partials(o_parts, l_parts, out, lse)
+    graph.replay()
     b.record(stream)
     b.synchronize()
     combine_us = a.elapsed_time(b) * 1e3 / steps
+    del graph
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the split-KV timing: {mla.status_string(st)} {word:#x}")
     exchange = x.batch * x.s_q * x.h_q * (512 + 1) * 4
-    return {"world": world, "rank_decode_us": rank_us, "rank_GB/s": rank_gbs,
-            "combine_us": combine_us, "exchange_bytes_per_rank": exchange,
+    total, _ = wl.algorithmic_work(x.seqlens, x.s_q, x.h_q, x.causal)
+    return {"world": world, "workload": f"b={x.batch} s_q=1 h_q=128 L={SPLIT_KV_LENGTHS[0]}",
+            "rank_decode_us": rank_us, "rank_GB/s": rank_gbs, "combine_us": combine_us,
+            "exchange_bytes_per_rank": exchange,
+            "GB/s_without_exchange": total / ((max(rank_us) + combine_us) * 1e-6) / 1e9,
             "note": f"each rank holds about 1/{world} of every sequence's pages; rank decodes "
                     "(fp32 partials, L2 flushed before each) and the merge of the gathered "
-                    "parts timed one after another on this GPU; the all-gather of "
-                    "exchange_bytes_per_rank per rank between GPUs is not timed"}
+                    "parts (replayed from a CUDA graph) timed one after another on this GPU; "
+                    "GB/s_without_exchange is "
+                    "the whole problem's bytes over the slowest rank plus the merge; the "
+                    "all-gather of exchange_bytes_per_rank per rank between GPUs is not "
+                    "timed"}
 
 
 def main():
@@ -459,7 +476,7 @@ def main():
     if st != 0:
         raise RuntimeError(f"device error in the cache append: {mla.status_string(st)} {word:#x}")
 
-    split_kv = time_split_kv(mla, x, flush, stream, args.steps) if args.split_kv > 1 else None
+    split_kv = time_split_kv(mla, flush, stream, args.steps, args.seed) if args.split_kv > 1 else None
 
     hbm_peak, tf_peak, peak_kind = peaks()
     avg_decode_s = statistics.mean(decode_ms) / 1e3

@@ -52,18 +52,32 @@ rank_combine_kernel(const RankCombineParams p) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         lse_row = mx + logf(sum);
-        for (int g = 0; g < p.parts; ++g) {
-            const float w = expf(p.lse_parts[g * lse_stride + lse_index] - lse_row);
-            if (w == 0.f) continue;       // an empty part (its O is 0 and must not be read as NaN)
-            const float4* src = reinterpret_cast<const float4*>(p.o_parts + g * o_stride +
-                                                                (size_t)row * kHeadDimV);
+        // parts four at a time, every load of a group in flight before its arithmetic
+        for (int g0 = 0; g0 < p.parts; g0 += 4) {
+            float w[4];
+            float4 x[4][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float4 x = src[lane + 32 * j];
-                acc[4 * j + 0] = fmaf(w, x.x, acc[4 * j + 0]);
-                acc[4 * j + 1] = fmaf(w, x.y, acc[4 * j + 1]);
-                acc[4 * j + 2] = fmaf(w, x.z, acc[4 * j + 2]);
-                acc[4 * j + 3] = fmaf(w, x.w, acc[4 * j + 3]);
+            for (int k = 0; k < 4; ++k) {
+                const int g = g0 + k;
+                w[k] = g < p.parts ? expf(p.lse_parts[g * lse_stride + lse_index] - lse_row) : 0.f;
+                // an empty part weighs 0 and its O (possibly NaN) is not read
+                if (w[k] != 0.f) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.o_parts + g * o_stride + (size_t)row * kHeadDimV);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) x[k][j] = src[lane + 32 * j];
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (w[k] == 0.f) continue;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[4 * j + 0] = fmaf(w[k], x[k][j].x, acc[4 * j + 0]);
+                    acc[4 * j + 1] = fmaf(w[k], x[k][j].y, acc[4 * j + 1]);
+                    acc[4 * j + 2] = fmaf(w[k], x[k][j].z, acc[4 * j + 2]);
+                    acc[4 * j + 3] = fmaf(w[k], x[k][j].w, acc[4 * j + 3]);
+                }
             }
         }
     }
