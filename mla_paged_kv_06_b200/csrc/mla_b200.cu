@@ -175,20 +175,6 @@ bool make_q_map(CUtensorMap* map, const void* q, size_t total_rows, int box_chun
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2D view of the page pool: [num_blocks * 64 rows][576 bf16], row stride 1152 bytes.
-bool make_pool_map(CUtensorMap* map, const void* kcache, int num_blocks, int box_cols,
-                   CUtensorMapSwizzle swz) {
-    EncodeTiledFn fn = encode_tiled_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)num_blocks * kBlock};
-    const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)kBlock};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kcache), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 mla_status validate_decode(const uint16_t* q, const uint16_t* kcache, int num_blocks,
                            const int32_t* block_table, int max_blocks, const int32_t* seqlens,
                            int batch, int s_q, int h_q, float scale, int causal,

@@ -36,13 +36,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
-// Arrive on a barrier of another CTA of the cluster (address from mapa), releasing this
-// thread's earlier shared::cluster stores to that CTA.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-                 : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -88,7 +81,7 @@ __device__ __forceinline__ void st_async_signal(uint32_t cluster_addr, uint32_t 
         ::"r"(cluster_addr), "r"(1u), "r"(cluster_bar) : "memory");
 }
 
-// Acquire at cluster scope: pairs with mbar_arrive_remote from the peer CTA.
+// Acquire at cluster scope: pairs with a release by the peer CTA (st.async, commit).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -169,27 +162,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 }
 
 // ---------------------------------------------------------------- TMA
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-        : "memory");
-}
-
-// The same load issued by either CTA of a 2-CTA pair, completing its bytes on a barrier
-// of the pair's even CTA (`bar` is that barrier's shared::cluster address): both CTAs'
-// halves of an operand then land on one barrier that the MMA issuer waits on.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
-                                                 uint32_t bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-        : "memory");
-}
-
 // 3-D tiled loads (a page viewed as {64 elements, rows, 128-byte chunks}): one
 // instruction moves several 8 KB swizzled tiles, which the TMA unit streams far faster
 // than the same bytes as separate 2-D boxes.
@@ -202,6 +174,9 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// The same load issued by either CTA of a 2-CTA pair, completing its bytes on a barrier
+// of the pair's even CTA (`bar` is that barrier's shared::cluster address): both CTAs'
+// halves of an operand then land on one barrier that the MMA issuer waits on.
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map,
                                                  uint32_t bar, int x, int y, int z) {
     asm volatile(
@@ -214,13 +189,6 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
 __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
     asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
                  ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z)
-                 : "memory");
-}
-
-// Prefetch a tile into L2 (no shared memory, no completion to wait for).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y)
                  : "memory");
 }
 
