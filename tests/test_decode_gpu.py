@@ -137,6 +137,31 @@ def test_more_units_than_clusters():
     compare(out, lse, *oracle_all(x), what="units > clusters")
 
 
+def test_thirty_thousand_sequences_sharing_a_small_pool():
+    # A batch too large for the scheduler's shared-memory table (its global-memory path
+    # runs), about 400 work sequences per unit, and a combine grid of 30,000 x 16 CTAs.
+    # The sequences map their pages into one 64-page pool (decode only reads the cache),
+    # so the inputs stay small. Sampled sequences, empty ones included, match the oracle.
+    lens = [(37 * i) % 701 for i in range(30000)]
+    batch, nblk_max, pool = len(lens), 11, 64
+    g = torch.Generator().manual_seed(74)
+    bt = torch.tensor([[(7 * b + 13 * j) % pool for j in range(nblk_max)] for b in range(batch)],
+                      dtype=torch.int32)
+    x = wl.DecodeInputs(
+        q=torch.randn((batch, 1, 1, 576), generator=g).to(torch.bfloat16),
+        kcache=torch.randn((pool, 64, 1, 576), generator=g).to(torch.bfloat16),
+        block_table=bt, seqlens=torch.tensor(lens, dtype=torch.int32),
+        scale=wl.DEFAULT_SCALE, causal=False, workload="custom", seed=74)
+    out, lse = run(x)
+    o = out.float().cpu().numpy()
+    assert np.isfinite(o).all()
+    idx = sorted({0, 1, 700, 701, 18947, batch - 1} | set(range(5, batch, 997)))
+    ref_out, ref_lse = oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale, False,
+                                     batch_indices=idx)
+    compare(out[idx], lse[idx], ref_out, ref_lse, what="30k sequences")
+    assert lens[0] == 0 and torch.all(out[0] == 0) and torch.isneginf(lse[0]).all()
+
+
 FULL = ["uniform", "v3", "spec", "skewed"]
 
 
