@@ -254,3 +254,65 @@ def test_planted_mistakes_are_caught(kind):
     mutant = _mutant_decode(kind)
     with pytest.raises(AssertionError):
         _check_golden(mutant)
+
+
+# ---------------------------------------------------------------------------------
+# decode_partial on its own: its output is the attention over an explicit token set, so
+# over the whole visible set of a row it must give what the brute-force loop gives for
+# that row. This pins the function independently of combine() (which only relates its
+# outputs to each other).
+
+def _partial_vs_bruteforce(partial_fn):
+    x = _small_case(12, [70, 130, 1], 2, 3, True)
+    bf_out, bf_lse = oracle.decode_bruteforce(x.q, x.kcache, x.block_table, x.seqlens,
+                                              x.scale, True)
+    kc = x.kcache.double().numpy()
+    for b, L in enumerate(x.seqlens.tolist()):
+        for i in range(x.s_q):
+            n = om.visible_tokens(L, x.s_q, i, True)
+            K = om.gather_tokens(kc, x.block_table[b].numpy(), max(n, 0))
+            o, l = partial_fn(x.q[b, i], K, x.scale)
+            np.testing.assert_allclose(o, bf_out[b, i], rtol=0, atol=1e-12)
+            if n > 0:
+                np.testing.assert_allclose(l, bf_lse[b, :, i], rtol=0, atol=1e-12)
+            else:
+                assert np.all(np.isneginf(l)) and np.all(o == 0)
+
+
+def test_decode_partial_matches_bruteforce_over_a_rows_visible_tokens():
+    _partial_vs_bruteforce(oracle.decode_partial)
+
+
+def test_decode_partial_matches_decode_on_a_workload_sequence():
+    x = _small_case(13, [300, 1000], 1, 8, False, poison=False, spare=0)
+    out, lse = oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale, False)
+    kc = x.kcache.double().numpy()
+    for b, L in enumerate([300, 1000]):
+        K = om.gather_tokens(kc, x.block_table[b].numpy(), L)
+        o, l = oracle.decode_partial(x.q[b, 0], K, x.scale)
+        np.testing.assert_allclose(o, out[b, 0], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l, lse[b, :, 0], rtol=0, atol=1e-12)
+
+
+def _mutant_partial(kind):
+    def partial(q_rows, K_rows, scale):
+        qq, K = om._f64(q_rows), om._f64(K_rows)
+        if K.shape[0] == 0:
+            return np.zeros((qq.shape[0], 512)), np.full(qq.shape[0], -np.inf)
+        S = scale * (qq @ K.T)
+        m = S.max(axis=1, keepdims=True)
+        E = np.exp(S - m)
+        lsum = E.sum(axis=1)
+        V = K[:, 64:] if kind == "v_last_dims" else K[:, :512]
+        o = E @ V
+        if kind != "no_normalise":
+            o = o / lsum[:, None]
+        lse = m[:, 0] + np.log(lsum) if kind != "lse_without_max" else np.log(lsum)
+        return o, lse
+    return partial
+
+
+@pytest.mark.parametrize("kind", ["v_last_dims", "no_normalise", "lse_without_max"])
+def test_planted_mistakes_in_decode_partial_are_caught(kind):
+    with pytest.raises(AssertionError):
+        _partial_vs_bruteforce(_mutant_partial(kind))
