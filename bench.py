@@ -39,6 +39,7 @@ kBlockRoom = 64                     # tokens per page
 LAUNCHES_PER_STEP = 3               # metadata, split kernel, combine kernel
 SPLIT_KV_WORLD = 4                  # ranks of the split-KV-across-devices measurement
 SPLIT_KV_LENGTHS = [65536] * 4      # its sequences: long contexts split over the ranks
+CONFIG_ORDER = ["tiny", "uniform", "v3", "spec", "skewed"]   # the `configs` entries
 
 
 def parse():
@@ -53,6 +54,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--split-kv", type=int, default=SPLIT_KV_WORLD,
                     help="ranks of the split-KV-across-devices timing (<= 1 skips it)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other workloads after the main one")
+    ap.add_argument("--config-cpu-seconds", type=float, default=4.0)
     return ap.parse_args()
 
 
@@ -295,6 +299,71 @@ def time_split_kv(mla, flush, stream, steps, seed):
                     "timed"}
 
 
+def roofline_fracs(nbytes, nflops, seconds, hbm_peak, tf_peak):
+    t_bytes = nbytes / (hbm_peak * 1e9)
+    t_flops = nflops / (tf_peak * 1e12)
+    return {"bound": "hbm" if t_bytes >= t_flops else "tensor",
+            "hbm_frac": t_bytes / seconds, "tensor_frac": t_flops / seconds,
+            "roofline_frac": max(t_bytes, t_flops) / seconds}
+
+
+def time_config(mla, name, seed, flush, stream, steps, warmup, hbm_peak, tf_peak,
+                cpu_seconds, with_cpu):
+    """One workload's decode timed the way the main measurement times it (L2 flushed,
+    untimed, before each step; metadata and decode call timed with CUDA events on the
+    launching stream), reported against its own roofline."""
+    x = wl.make_workload(name, seed=seed)
+    d = dict(q=x.q.cuda(), kcache=x.kcache.cuda(), block_table=x.block_table.cuda(),
+             seqlens=x.seqlens.cuda())
+    nsm = mla.default_num_sms()
+    meta = torch.empty(mla.mla_metadata_ints(nsm), dtype=torch.int32, device="cuda")
+    ns = torch.empty(mla.mla_num_splits_len(x.batch, x.h_q, x.s_q), dtype=torch.int32,
+                     device="cuda")
+    ws = torch.empty(mla.mla_workspace_bytes(x.batch, x.h_q, x.s_q, nsm), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((x.batch, x.s_q, x.h_q, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
+    for _ in range(max(warmup, 3)):
+        flush.zero_()
+        mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
+        mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
+                           x.causal, meta, ns, ws, out, lse)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        e0, e1, e2 = ev[k]
+        e0.record(stream)
+        mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
+        e1.record(stream)
+        mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
+                           x.causal, meta, ns, ws, out, lse)
+        e2.record(stream)
+    torch.cuda.synchronize()
+    st, word = mla.mla_get_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in {name}: {mla.status_string(st)} {word:#x}")
+    step_ms = [a.elapsed_time(c) for a, _, c in ev]
+    decode_ms = [b.elapsed_time(c) for _, b, c in ev]
+    nbytes, nflops = wl.algorithmic_work(x.seqlens, x.s_q, x.h_q, x.causal)
+    t = statistics.mean(decode_ms) / 1e3
+    rows = x.s_q * x.h_q
+    entry = {"workload": workload_config(x, name)["workload"], "batch": x.batch,
+             "s_q": x.s_q, "h_q": x.h_q, "total_tokens": int(x.seqlens.sum()),
+             "kernel": "1-CTA (rows <= 64)" if rows <= 64 else "2-CTA pairs",
+             "us_per_call": statistics.median(step_ms) * 1e3,
+             "us_per_call_decode": statistics.median(decode_ms) * 1e3,
+             "GB/s": nbytes / t / 1e9, "TFLOPS": nflops / t / 1e12,
+             "algorithmic_bytes": nbytes, "algorithmic_flops": nflops,
+             "roofline": roofline_fracs(nbytes, nflops, t, hbm_peak, tf_peak)}
+    if with_cpu:
+        entry["cpu_baseline"] = cpu_baseline(x, cpu_seconds)
+    del d, ws, out, lse
+    torch.cuda.empty_cache()
+    return entry
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -479,6 +548,16 @@ def main():
     split_kv = time_split_kv(mla, flush, stream, args.steps, args.seed) if args.split_kv > 1 else None
 
     hbm_peak, tf_peak, peak_kind = peaks()
+    # every workload of the benchmark in the same run, each against its own roofline
+    configs = {}
+    if not args.no_configs:
+        for name in CONFIG_ORDER:
+            if name == args.workload:
+                continue
+            configs[name] = time_config(
+                mla, name, rank_seed(args.seed, rank), flush, stream, args.steps, args.warmup,
+                hbm_peak, tf_peak, args.config_cpu_seconds,
+                with_cpu=rank == 0 and world == 1 and not args.no_cpu_baseline)
     avg_decode_s = statistics.mean(decode_ms) / 1e3
     achieved_gbs = nbytes / avg_decode_s / 1e9
     achieved_tf = nflops / avg_decode_s / 1e12
@@ -542,6 +621,19 @@ def main():
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x, args.cpu_seconds)
+    if not args.no_configs:
+        main_entry = {"workload": line["config"]["workload"], "batch": x.batch, "s_q": x.s_q,
+                      "h_q": x.h_q, "total_tokens": int(x.seqlens.sum()),
+                      "kernel": "1-CTA (rows <= 64)" if x.s_q * x.h_q <= 64 else "2-CTA pairs",
+                      "us_per_call": line["us_per_call"],
+                      "us_per_call_decode": line["us_per_call_decode"],
+                      "GB/s": achieved_gbs, "TFLOPS": achieved_tf,
+                      "algorithmic_bytes": nbytes, "algorithmic_flops": nflops,
+                      "roofline": roofline_fracs(nbytes, nflops, avg_decode_s, hbm_peak, tf_peak)}
+        if "cpu_baseline" in line:
+            main_entry["cpu_baseline"] = line["cpu_baseline"]
+        line["configs"] = {n: (main_entry if n == args.workload else configs[n])
+                           for n in CONFIG_ORDER}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
@@ -551,7 +643,7 @@ def main():
 
 
 # Bumped whenever the split kernel changes, so stale ncu traffic is never reported.
-KERNEL_REV = "pair-4"
+KERNEL_REV = "pair-5"
 
 if __name__ == "__main__":
     sys.exit(main())

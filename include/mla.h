@@ -97,10 +97,12 @@ size_t mla_num_splits_len(int batch, int h_q, int s_q);
  * for sizes the library rejects. */
 size_t mla_workspace_bytes(int batch, int h_q, int s_q, int num_sms);
 
-/* Work units (pairs of SMs) a schedule for `num_sms` uses on the current device:
- * min(num_sms / 2, co-resident 2-CTA clusters of the decode kernel), at least 1.
- * Returns a negative mla_status on failure. */
-int mla_num_work_units(int num_sms);
+/* Work units a schedule for `num_sms` uses on the current device for these shapes.
+ * Sequences of at most 64 query rows (s_q * h_q <= 64) run on the 1-CTA kernel, one unit
+ * per SM: min(num_sms, co-resident CTAs). Larger ones run on the 2-CTA kernel, one unit
+ * per pair of SMs: min(num_sms / 2, co-resident 2-CTA clusters). At least 1. Returns a
+ * negative mla_status on failure or for unsupported shapes. */
+int mla_num_work_units(int num_sms, int h_q, int s_q);
 
 /*
  * Split-KV tile scheduler (variable-length batches: FlashMLA release article,
@@ -126,9 +128,11 @@ mla_status mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q,
                             int32_t* metadata, int32_t* num_splits, void* stream);
 
 /*
- * Decode attention (see the operation above). Runs the sm_100a split kernel
- * (TMA page gather -> tcgen05 QK^T and PV with TMEM accumulators -> fp32 online
- * softmax with tail and causal masks) and then the LSE-weighted combine kernel.
+ * Decode attention (see the operation above). Runs an sm_100a split kernel (TMA page
+ * gather -> tcgen05 QK^T and PV with TMEM accumulators -> fp32 online softmax with tail
+ * and causal masks) and then the LSE-weighted combine kernel. Sequences of at most 64
+ * query rows (s_q * h_q <= 64) use a 1-CTA kernel with a transposed PV (O^T = V^T P^T);
+ * larger ones use 2-CTA pairs that split each 128-row tile between two SMs.
  *
  *   q, kcache, block_table, seqlens, out, lse: device buffers in the layout above;
  *     q, kcache and out must be 16-byte aligned.
@@ -165,12 +169,16 @@ mla_status mla_decode_fwd(const uint16_t* q, const uint16_t* kcache, int num_blo
  *
  *   Limit: sizes whose worst-case partials exceed the array, over every schedule the
  *     current device can run (one [128][512] fp32 tile per work sequence plus one per
- *     work unit), return MLA_ERR_WORKSPACE_TOO_SMALL before anything is launched. On a
- *     148-SM B200 that admits batch * ceil(s_q*h_q/128) up to 181. Larger batches must
- *     use mla_decode_fwd with a workspace.
+ *     work unit), return MLA_ERR_WORKSPACE_TOO_SMALL before anything is launched. The
+ *     array holds 255 tiles. On a 148-SM B200 that admits batch * ceil(s_q*h_q/128) up
+ *     to 181 when s_q*h_q > 64 (74 units) and batch up to 107 when s_q*h_q <= 64 (148
+ *     units). Larger batches must use mla_decode_fwd with a workspace.
  *   First call: the first call on each device, with that device current, looks up the
  *     array's device address (cudaGetSymbolAddress) and does mla_decode_fwd's one-time
- *     kernel set-up. Make that first call before any stream capture begins.
+ *     kernel set-up. Make that first call before any stream capture begins. The address
+ *     is cached for the life of the process: after cudaDeviceReset (or any other
+ *     teardown of the device's primary context) this entry point must not be called
+ *     again in that process.
  *   Sharing: every call on a device, from any stream or host thread, uses the same
  *     array, which keeps the partials of the last call. Nothing in it has to start at
  *     zero: a call reads only partials it has written itself.
@@ -284,6 +292,26 @@ mla_status mla_kv_append_fp8(const uint16_t* kv_new, int s_new, const int32_t* b
  * word: bits 0-7 the error kind, the rest where it arose.
  */
 mla_status mla_get_last_device_error(void* stream, uint32_t* detail);
+
+/*
+ * What MLA_ERR_DEVICE_TIMEOUT leaves behind: a pipeline wait ran out of its limit (2 s by
+ * default), which only a broken input, a broken kernel or a stalled device can cause.
+ * The CTA that gave up stops every role, waits (again with the limit) for the MMAs it
+ * issued and, in the 1-CTA kernel, for its own copies, then frees its TMEM and exits;
+ * in the 2-CTA kernel a copy still in flight is only given a fixed 50 us to land. Treat
+ * the results of that call as garbage and, if timeouts repeat, the device context as
+ * suspect.
+ *
+ * Test hook for the bounded waits (not for production use). With stall = 1, every
+ * decode kernel launched afterwards (mla_decode_fwd and its variants) has its loader wait
+ * on a barrier that nothing completes, before it issues any copy, so every wait of the
+ * kernel gives up after `wait_limit_ns`: the kernel records MLA_ERR_DEVICE_TIMEOUT and
+ * exits normally with nothing in flight, and the device stays usable. stall = 0 restores
+ * normal decoding. wait_limit_ns sets the limit of every wait (0 restores the default
+ * of 2 s). Both settings live on the current device, where the call writes them
+ * synchronously; every later launch on that device reads them.
+ */
+mla_status mla_test_set_stall(int stall, unsigned long long wait_limit_ns);
 
 /*
  * Host-side copy of the scheduler, for tests and for callers that plan on the CPU:

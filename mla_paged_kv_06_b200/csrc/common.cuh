@@ -47,6 +47,11 @@ __device__ __forceinline__ int visible_tokens(int L, int s_q, int i, int causal)
 
 // Device error word of the library (one translation unit includes this header).
 __device__ uint32_t g_mla_error = 0;
+// Limit of every pipeline wait, in ns, and the stall test hook (mla_test_set_stall sets
+// both on the current device; kept out of DecodeParams, whose size the 2-CTA kernel's
+// register budget feels).
+__device__ unsigned long long g_mla_wait_limit_ns = 2000000000ull;
+__device__ int g_mla_debug_stall = 0;
 
 namespace mla {
 

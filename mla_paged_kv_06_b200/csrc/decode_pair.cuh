@@ -54,6 +54,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "items.cuh"
 #include "ptx.cuh"
 
 namespace mla {
@@ -65,7 +66,6 @@ constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
 constexpr int kPrefetchSteps = 1;                    // L2 prefetch distance in steps (fastest of 0-4)
 constexpr float kRescaleLog2 = 8.0f;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s per wait, then give up
 
 constexpr uint32_t kBoxBytes = 64 * 128;             // 64 rows x 64 bf16, SW128
 constexpr int kBoxesPerPage = 9;                     // 8 latent + 1 rope
@@ -80,8 +80,8 @@ constexpr uint32_t kOffQs = kOffK + 2 * kStageBytes;
 constexpr uint32_t kOffP = kOffQs + kQsBoxes * kBoxBytes;
 constexpr uint32_t kOffMax = kOffP + 2 * kPBytes;             // [2 grp][2 par][2 half][64] f32
 constexpr uint32_t kOffMref = kOffMax + 2 * 2 * 2 * 64 * 4;   // [2 par][64] f32
-constexpr uint32_t kOffLsum = kOffMref + 2 * 64 * 4;          // [2 grp][2 half][64] f32
-constexpr uint32_t kOffBar = kOffLsum + 2 * 2 * 64 * 4;
+constexpr uint32_t kOffLsum = kOffMref + 2 * 64 * 4;          // [2 sum][2 grp][2 half][64] f32
+constexpr uint32_t kOffBar = kOffLsum + 2 * 2 * 2 * 64 * 4;
 enum : uint32_t {
     kBarKFull = 0,                  // [2] both pages of the step landed (CTA 0's copy used)
     kBarQkDone = kBarKFull + 2,     // [2] QK of the step done (both CTAs)
@@ -95,7 +95,8 @@ enum : uint32_t {
     kBarMref = kBarMaxX + 2,        // [2 groups] reference max of the step posted
     kBarLsum = kBarMref + 2,        // both groups posted their row sums
     kBarDrain = kBarLsum + 1,       // the MMA issuer's last commit
-    kNumBars = kBarDrain + 1
+    kBarStall = kBarDrain + 1,      // never completes (the timeout test hook waits on it)
+    kNumBars = kBarStall + 1
 };
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem base, abort flag, sink word
 // bytes CTA 1 signals per phase: one 4-byte store per softmax warp that arrives
@@ -103,7 +104,7 @@ constexpr uint32_t kPReadyTx = 4 * 4;
 constexpr uint32_t kQReadyTx = 8 * 4;
 constexpr uint32_t kOFreeTx = 8 * 4;
 constexpr uint32_t kQBytes = 9 * kBoxBytes;             // 64 q rows x 576 dims
-constexpr uint32_t kSmemBytes = kOffMisc + 16;
+constexpr uint32_t kSmemBytes = kOffMisc + 24;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;      // room to align the base to 1 KB
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
 
@@ -127,6 +128,10 @@ struct Shared {
     }
     __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + kOffMisc); }
     __device__ uint32_t sink() const { return base_u32 + kOffMisc + 12; }
+    // ns a wait may last before the kernel gives up (read only on the slow path)
+    __device__ uint64_t wait_limit() const {
+        return *reinterpret_cast<volatile uint64_t*>(base + kOffMisc + 16);
+    }
 };
 
 // Bounded wait (as in every kernel of the library): false if the phase does not complete
@@ -142,7 +147,7 @@ __device__ __forceinline__ bool wait_bar(const Shared& sh, uint32_t bar, uint32_
             return true;
         if ((it & 255u) == 255u) {
             if (*sh.abort_flag()) return false;
-            if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+            if (ptx::globaltimer() - t0 > sh.wait_limit()) {
                 *sh.abort_flag() = 1;
                 record_error(kErrTimeout, where);
                 return false;
@@ -160,64 +165,6 @@ __device__ __forceinline__ bool warp_wait_bar(const Shared& sh, uint32_t bar, ui
     return __all_sync(0xffffffffu, ok);
 }
 
-// One piece of work: pages [k_lo, k_hi) of work sequence v.
-struct Item {
-    int v, b, t, L, k_lo, k_hi, chunk, n_chunks, part;
-    __device__ int steps() const { return (k_hi - k_lo + 1) >> 1; }
-};
-
-// Iterates the items of every unit this cluster owns, in the same order for all roles.
-struct ItemIter {
-    const DecodeParams& p;
-    int u, num_units, V, step;
-    int v, v_end, k_begin, k_end, chunk_begin, v_begin;
-    __device__ ItemIter(const DecodeParams& pp, int first_unit, int unit_step)
-        : p(pp), u(first_unit - unit_step), step(unit_step) {
-        num_units = p.metadata[0];
-        V = p.batch * p.tiles;
-        v = 1;
-        v_end = 0;
-    }
-    __device__ bool next(Item& it) {
-        for (;;) {
-            if (v > v_end || v >= V) {
-                u += step;
-                if (u >= num_units) return false;
-                const int32_t* m = p.metadata + kMetaInts * (u + 1);
-                v_begin = m[0]; k_begin = m[1]; v_end = m[2]; k_end = m[3]; chunk_begin = m[4];
-                v = v_begin;
-                continue;
-            }
-            const int vv = v++;
-            it.v = vv;
-            it.b = vv % p.batch;
-            it.t = vv / p.batch;
-            it.L = checked_seqlen(p, it.b);
-            const int nblk = pages_of(it.L);
-            it.k_lo = vv == v_begin ? k_begin : 0;
-            it.k_hi = vv == v_end ? k_end : nblk;
-            if (it.k_hi > nblk) it.k_hi = nblk;
-            if (it.k_lo >= it.k_hi) continue;
-            it.chunk = vv == v_begin ? chunk_begin : 0;
-            it.n_chunks = p.num_splits[vv + 1] - p.num_splits[vv];
-            it.part = p.num_splits[vv] + it.chunk;
-            return true;
-        }
-    }
-};
-
-// First pool row of logical page k of sequence b, or the row just past the pool (a box
-// there is read as zeros) when the page is outside [k_lo, k_hi) or its id is invalid.
-__device__ __forceinline__ int page_row(const DecodeParams& p, int b, int k, int k_hi) {
-    if (k >= k_hi) return p.num_blocks * kBlock;
-    const int pid = p.block_table[(size_t)b * p.max_blocks + k];
-    if (pid < 0 || pid >= p.num_blocks) {
-        record_error(kErrBadInput, 0x800000u | ((uint32_t)b & 0x7fffffu));
-        return p.num_blocks * kBlock;
-    }
-    return pid * kBlock;
-}
-
 // ------------------------------------------------------------------ producer (warp 8)
 // tm_page: box {64, 64 rows, 9 chunks} (a whole page); tm_pair: box {64, 64 rows, 2}.
 // Step S uses stage S % 2. This CTA's page of the step is loaded whole once PV of step
@@ -229,6 +176,13 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
                                              const CUtensorMap* tm_page, const CUtensorMap* tm_pair,
                                              const CUtensorMap* tm_q4, const CUtensorMap* tm_q5,
                                              uint32_t crank) {
+    if (g_mla_debug_stall) {
+        // test hook: wait on a barrier nothing completes, before any copy is issued; the
+        // wait gives up after the limit, so every role of the CTA stops with nothing in
+        // flight and the timeout is recorded
+        wait_bar<false>(sh, sh.bar(kBarStall), 0, 0x13u);
+        return;
+    }
     ItemIter iter(p, (int)ptx::cluster_id_x(), (int)ptx::nclusters_x());
     Item it;
     bool have = iter.next(it);
@@ -329,7 +283,7 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             if (*sh.abort_flag()) return;
             const uint64_t now = ptx::globaltimer();
             if (idle == 1024u) t0 = now;
-            else if (now - t0 > kWaitLimitNs) {
+            else if (now - t0 > sh.wait_limit()) {
                 *sh.abort_flag() = 1;
                 record_error(kErrTimeout, 0x10u);
                 return;
@@ -347,6 +301,9 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
 // ------------------------------------------------------------------ MMA issuer (CTA 0)
 // S of step S goes to TMEM buffer S % 2, free once PV of step S - 2 was issued (its P
 // was written after the softmax had read that S).
+// K-steps [k0, k1) of the 36 (16 dims each) of QK for step S; the part that ends at 36
+// commits the step's QkDone.
+template <int k0, int k1>
 __device__ __forceinline__ void issue_qk(const Shared& sh, uint32_t tmem, uint32_t S) {
     const uint32_t b = S & 1u;
     ptx::tc_fence_after();
@@ -354,18 +311,17 @@ __device__ __forceinline__ void issue_qk(const Shared& sh, uint32_t tmem, uint32
     const uint32_t st = sh.stage(b);
     const uint32_t qs = sh.base_u32 + kOffQs;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {                 // latent dims [0,256): Q from TMEM
+    for (int k = k0; k < k1; ++k) {
         const uint64_t bdesc = ptx::smem_desc(st + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024, 2);
-        ptx::mma_ts_pair(d, tmem + kColQ + 8 * k, bdesc, kIdescQK, k > 0 ? 1u : 0u);
+        if (k < 16) {                              // latent dims [0,256): Q from TMEM
+            ptx::mma_ts_pair(d, tmem + kColQ + 8 * k, bdesc, kIdescQK, k > 0 ? 1u : 0u);
+        } else {                                   // dims [256,576): Q from shared memory
+            const uint64_t adesc =
+                ptx::smem_desc(qs + ((k - 16) >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024, 2);
+            ptx::mma_ss_pair(d, adesc, bdesc, kIdescQK, 1u);
+        }
     }
-#pragma unroll
-    for (int k = 16; k < 36; ++k) {                // dims [256,576): Q from shared memory
-        const uint64_t adesc =
-            ptx::smem_desc(qs + ((k - 16) >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024, 2);
-        const uint64_t bdesc = ptx::smem_desc(st + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024, 2);
-        ptx::mma_ss_pair(d, adesc, bdesc, kIdescQK, 1u);
-    }
-    ptx::mma_commit_pair(sh.bar(kBarQkDone + b), kBothCtas);
+    if constexpr (k1 == 36) ptx::mma_commit_pair(sh.bar(kBarQkDone + b), kBothCtas);
 }
 
 // O += P V for step S; `first` starts the item's accumulation.
@@ -421,14 +377,14 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Shared& sh,
                 idle = 0;
             } else if (qk < n && qk < pv + 2 &&
                        ptx::mbar_test_wait_cluster(sh.bar(kBarKFull + (Sq & 1u)), (Sq >> 1) & 1u)) {
-                issue_qk(sh, tmem, Sq);
+                issue_qk<0, 36>(sh, tmem, Sq);
                 ++qk;
                 idle = 0;
             } else if ((++idle & 1023u) == 0) {
                 if (*sh.abort_flag()) { ok = false; break; }
                 const uint64_t now = ptx::globaltimer();
                 if (idle == 1024u) t0 = now;
-                else if (now - t0 > kWaitLimitNs) {
+                else if (now - t0 > sh.wait_limit()) {
                     *sh.abort_flag() = 1;
                     record_error(kErrTimeout, 0x24u);
                     ok = false;
@@ -456,13 +412,16 @@ struct SoftmaxCtx {
 };
 
 struct RowState {
-    float m_used;     // reference the sum is relative to (-inf: nothing yet)
-    float l_sum;      // sum of 2^(s - m_used) over this thread's tokens
+    float m_used;     // reference the sums are relative to (-inf: nothing yet)
+    float l_sum;      // sum of 2^(s - m_used) over this thread's tokens (for the lse)
+    float l_rnd;      // the same sum of the bf16-rounded values PV multiplies (normalises O)
 };
 
 __device__ __forceinline__ void rebase(RowState& st, float m) {
     if (m != st.m_used) {
-        st.l_sum = st.m_used == -INFINITY ? 0.f : st.l_sum * ptx::ex2_ftz(st.m_used - m);
+        const float f = st.m_used == -INFINITY ? 0.f : ptx::ex2_ftz(st.m_used - m);
+        st.l_sum *= f;
+        st.l_rnd *= f;
         st.m_used = m;
     }
 }
@@ -549,17 +508,24 @@ __device__ __forceinline__ bool softmax_step(const DecodeParams& p, const Shared
         ptx::tmem_wait_st();
     }
     uint32_t pk[32];
-    float rs0 = 0.f, rs1 = 0.f;
+    float rs0 = 0.f, rs1 = 0.f, rr0 = 0.f, rr1 = 0.f;
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
         const float p0 = ptx::ex2_ftz(s[2 * q]);
         const float p1 = ptx::ex2_ftz(s[2 * q + 1]);
         rs0 += p0;
         rs1 += p1;
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        pk[q] = *reinterpret_cast<uint32_t*>(&h2);
+        // O is normalised by the sum of the bf16 values PV multiplies, so it is a weighted
+        // mean of V rows whose weights sum to one: a dominant token's rounding (its P may
+        // be up to 2^kRescaleLog2, not 1) then cancels instead of scaling the output. The
+        // lse keeps the exact sum.
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        rr0 += __low2float(h2);
+        rr1 += __high2float(h2);
+        pk[q] = *reinterpret_cast<const uint32_t*>(&h2);
     }
     st.l_sum += rs0 + rs1;
+    st.l_rnd += rr0 + rr1;
 
     // P buffer b is free once PV of step S-2 has completed
     if (S >= 2 && !warp_wait_bar<false>(sh, sh.bar(kBarPvDone + b), ((S - 2) >> 1) & 1u, 0x35u))
@@ -627,14 +593,16 @@ __device__ __forceinline__ bool epilogue(const DecodeParams& p, const Shared& sh
     rebase(e.st, m_fin);
     float* lsum = sh.fptr(kOffLsum);
     lsum[(c.grp * 2 + c.half) * 64 + row] = e.st.l_sum;
+    lsum[256 + (c.grp * 2 + c.half) * 64 + row] = e.st.l_rnd;
     ptx::mbar_arrive(sh.bar(kBarLsum));
     if (!warp_wait_bar<false>(sh, sh.bar(kBarLsum), epi_index & 1u, 0x37u)) return false;
     if (!warp_wait_bar<false>(sh, sh.bar(kBarPvDone + (Sl & 1u)), (Sl >> 1) & 1u, 0x34u)) return false;
     ptx::tc_fence_after();
     volatile float* vl = lsum;
     const float l_tot = (vl[row] + vl[64 + row]) + (vl[128 + row] + vl[192 + row]);
+    const float l_rnd = (vl[256 + row] + vl[320 + row]) + (vl[384 + row] + vl[448 + row]);
     const bool empty = !(l_tot > 0.f);
-    const float inv = empty ? 0.f : 1.f / l_tot;
+    const float inv = empty ? 0.f : 1.f / l_rnd;
     const float lse2 = empty ? -INFINITY : m_fin + __log2f(l_tot);
     const Item& it = e.it;
     const bool final_out = it.n_chunks == 1;
@@ -787,7 +755,7 @@ __device__ __forceinline__ void run_softmax(const DecodeParams& p, const Shared&
             signal_leader(sh, crank, kBarOFree);
         }
 
-        RowState st{-INFINITY, 0.f};
+        RowState st{-INFINITY, 0.f, 0.f};
         const uint32_t n = (uint32_t)it.steps();
         const uint32_t S0 = S;
         bool ok = true;
@@ -838,7 +806,9 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
         ptx::mbar_init(sh.bar(kBarOFree), 8 + 1);               // CTA 0's warps + arming
         ptx::mbar_init(sh.bar(kBarLsum), kSoftmaxThreads);
         ptx::mbar_init(sh.bar(kBarDrain), 1);
+        ptx::mbar_init(sh.bar(kBarStall), 1);
         *sh.abort_flag() = 0;
+        *reinterpret_cast<volatile uint64_t*>(sh.base + kOffMisc + 16) = g_mla_wait_limit_ns;
         ptx::fence_mbarrier_init_cluster();
         // arm the first phases of the barriers CTA 1 signals with byte counts
         ptx::mbar_arrive_expect_tx(sh.bar(kBarPReady + 0), kPReadyTx);

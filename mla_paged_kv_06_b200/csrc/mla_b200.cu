@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "decode_simt.cuh"
 #include "decode_pair.cuh"
+#include "decode_solo.cuh"
 #include "metadata.cuh"
 #include "rank_combine.cuh"
 #include "sched.cuh"
@@ -40,11 +41,23 @@ bool shape_ok(int batch, int h_q, int s_q) {
            s_q >= 1 && s_q <= MLA_MAX_S_Q && h_q * s_q <= MLA_MAX_ROWS;
 }
 
-int units_bound(int num_sms) { return num_sms / 2 < 1 ? 1 : num_sms / 2; }
+// Query rows per sequence up to which the 1-CTA kernel (decode_solo.cuh) runs; above it
+// the 2-CTA kernel (decode_pair.cuh) splits 128-row tiles over two SMs.
+constexpr int kSoloMaxRows = 64;
+
+bool use_solo(int h_q, int s_q) { return h_q * s_q <= kSoloMaxRows; }
+
+// Work units a schedule for num_sms SMs may use, before the device cap: one per SM for
+// the 1-CTA kernel, one per SM pair for the 2-CTA kernel.
+int units_bound(int num_sms, int h_q, int s_q) {
+    const int u = use_solo(h_q, s_q) ? num_sms : num_sms / 2;
+    return u < 1 ? 1 : u;
+}
 
 size_t max_chunks_for(int batch, int h_q, int s_q, int num_sms) {
-    return (size_t)batch * num_tiles(h_q, s_q) + (size_t)units_bound(num_sms);
+    return (size_t)batch * num_tiles(h_q, s_q) + (size_t)units_bound(num_sms, h_q, s_q);
 }
+
 
 constexpr size_t kChunkBytes = (size_t)kTileRows * 4 + (size_t)kTileRows * kHeadDimV * 4;
 
@@ -55,6 +68,11 @@ size_t ws_capacity(size_t bytes) {
 }
 
 size_t ws_o_offset(size_t cap) { return align_up(kWsHeader + cap * kTileRows * 4, kAlign); }
+
+// Workspace bytes that hold `cap` partial slots.
+size_t workspace_bytes_for(size_t cap) {
+    return ws_o_offset(cap) + cap * kTileRows * kHeadDimV * 4 + kAlign;
+}
 
 // Opt the split kernel into its shared-memory footprint (once per device).
 bool prepare_split_kernel(int dev) {
@@ -126,6 +144,54 @@ int device_pairs(int dev) {
     return pairs;
 }
 
+template <int kN>
+bool prepare_solo_kernel(int dev) {
+    static std::mutex mu;
+    static std::vector<char> done;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)done.size() <= dev) done.resize(dev + 1, 0);
+    if (done[dev]) return true;
+    if (cudaFuncSetAttribute(solo::decode_kernel<kN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)solo::Cfg<kN>::kSmemAlloc) != cudaSuccess)
+        return false;
+    done[dev] = 1;
+    return true;
+}
+
+// CTAs of the 1-CTA kernel that can be co-resident on a device (cached per device): one
+// per SM, as its shared memory and TMEM allow no second. A schedule never uses more
+// units than this, so every unit runs in one wave.
+int device_solo_ctas(int dev) {
+    static std::mutex mu;
+    static std::vector<int> cache;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if ((int)cache.size() > dev && cache[dev] > 0) return cache[dev];
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return -1;
+    int ctas = sms < 1 ? 1 : sms;
+    if (prepare_solo_kernel<64>(dev)) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, solo::decode_kernel<64>,
+                                                          solo::kThreads,
+                                                          solo::Cfg<64>::kSmemAlloc) == cudaSuccess &&
+            per_sm >= 1 && per_sm * sms < ctas)
+            ctas = per_sm * sms;
+        cudaGetLastError();
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+    cache[dev] = ctas;
+    return ctas;
+}
+
+// Units of every schedule the current device can run for these shapes.
+int device_units(int dev, int h_q, int s_q) {
+    return use_solo(h_q, s_q) ? device_solo_ctas(dev) : device_pairs(dev);
+}
+
 // cuTensorMapEncodeTiled from the driver, found at run time so the library does not
 // link libcuda (it must load on machines without a GPU driver).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -162,13 +228,14 @@ bool make_page_map(CUtensorMap* map, const void* kcache, int num_blocks, int box
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The same 3-D view of q ([total rows][576] bf16): box {64, 64 rows, box_chunks}.
-bool make_q_map(CUtensorMap* map, const void* q, size_t total_rows, int box_chunks) {
+// The same 3-D view of q ([total rows][576] bf16): box {64, box_rows, box_chunks}.
+bool make_q_map(CUtensorMap* map, const void* q, size_t total_rows, int box_chunks,
+                int box_rows = 64) {
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {64, (cuuint64_t)total_rows, (cuuint64_t)(kHeadDim / 64)};
     const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, 128};
-    const cuuint32_t box[3] = {64, 64, (cuuint32_t)box_chunks};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_chunks};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -246,9 +313,53 @@ void* noalloc_scratch(int dev) {
 }
 
 mla_status launch_combine(const DecodeParams& p, cudaStream_t s) {
-    dim3 grid(p.batch * p.tiles, kTileRows / kCombineRowsPerCta);
+    // one warp per row of a tile; a tile of a sequence with fewer rows needs fewer CTAs
+    const int tile_rows = p.rows < kTileRows ? p.rows : kTileRows;
+    dim3 grid(p.batch * p.tiles, (tile_rows + kCombineRowsPerCta - 1) / kCombineRowsPerCta);
     combine_kernel<<<grid, kCombineThreads, 0, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+template <int kN>
+mla_status launch_solo(const DecodeParams& p, const void* q, const void* kcache, int num_blocks,
+                       int ctas, int dev, cudaStream_t s) {
+    if (!prepare_solo_kernel<kN>(dev)) return MLA_ERR_CUDA;
+    CUtensorMap tm_page, tm_q;
+    if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
+        !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
+        return MLA_ERR_CUDA;
+    solo::decode_kernel<kN><<<ctas, solo::kThreads, solo::Cfg<kN>::kSmemAlloc, s>>>(p, tm_page, tm_q);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// The split kernel for these shapes (1-CTA up to 64 rows per sequence, else 2-CTA
+// pairs), then the combine. `p` is complete; q and kcache are its tensors.
+mla_status launch_decode(const DecodeParams& p, const void* q, const void* kcache,
+                         int num_blocks, cudaStream_t s) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    mla_status st = MLA_OK;
+    if (p.rows <= kSoloMaxRows) {
+        const int ctas = device_solo_ctas(dev);
+        if (ctas < 1) return MLA_ERR_CUDA;
+        st = p.rows <= 16 ? launch_solo<16>(p, q, kcache, num_blocks, ctas, dev, s)
+           : p.rows <= 32 ? launch_solo<32>(p, q, kcache, num_blocks, ctas, dev, s)
+                          : launch_solo<64>(p, q, kcache, num_blocks, ctas, dev, s);
+    } else {
+        const int pairs = device_pairs(dev);
+        if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
+        CUtensorMap tm_page, tm_pair, tm_q4, tm_q5;
+        const size_t q_rows = (size_t)p.batch * p.rows;
+        if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
+            !make_page_map(&tm_pair, kcache, num_blocks, 2) ||
+            !make_q_map(&tm_q4, q, q_rows, 4) || !make_q_map(&tm_q5, q, q_rows, 5))
+            return MLA_ERR_CUDA;
+        pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair,
+                                                                              tm_q4, tm_q5);
+        st = cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    }
+    if (st != MLA_OK) return st;
+    return launch_combine(p, s);
 }
 
 // mla_decode_fwd and mla_decode_fwd_partial: bf16 `out` or fp32 `out_f32` (one is null).
@@ -267,21 +378,7 @@ mla_status decode_tc(const uint16_t* q, const uint16_t* kcache, int num_blocks,
                                  batch, s_q, h_q, scale, causal, metadata, num_splits,
                                  workspace, workspace_bytes, out, lse);
     p.out_f32 = out_f32;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-    const int pairs = device_pairs(dev);
-    if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
-    CUtensorMap tm_page, tm_pair, tm_q4, tm_q5;
-    const size_t q_rows = (size_t)batch * s_q * h_q;
-    if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
-        !make_page_map(&tm_pair, kcache, num_blocks, 2) ||
-        !make_q_map(&tm_q4, q, q_rows, 4) || !make_q_map(&tm_q5, q, q_rows, 5))
-        return MLA_ERR_CUDA;
-    cudaStream_t s = (cudaStream_t)stream;
-    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair,
-                                                                          tm_q4, tm_q5);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-    return launch_combine(p, s);
+    return launch_decode(p, q, kcache, num_blocks, (cudaStream_t)stream);
 }
 
 }  // namespace
@@ -312,26 +409,35 @@ size_t mla_num_splits_len(int batch, int h_q, int s_q) {
 
 size_t mla_workspace_bytes(int batch, int h_q, int s_q, int num_sms) {
     if (!shape_ok(batch, h_q, s_q) || num_sms < 1) return 0;
-    const size_t cap = max_chunks_for(batch, h_q, s_q, num_sms);
-    return ws_o_offset(cap) + cap * kTileRows * kHeadDimV * 4 + kAlign;
+    return workspace_bytes_for(max_chunks_for(batch, h_q, s_q, num_sms));
 }
 
-int mla_num_work_units(int num_sms) {
+int mla_num_work_units(int num_sms, int h_q, int s_q) {
     if (num_sms < 1) return MLA_ERR_INVALID_ARG;
+    if (h_q < 1 || s_q < 1 || h_q > MLA_MAX_H_Q || s_q > MLA_MAX_S_Q || h_q * s_q > MLA_MAX_ROWS)
+        return MLA_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-    const int pairs = device_pairs(dev);
-    if (pairs < 1) return MLA_ERR_CUDA;
-    int u = num_sms / 2;
-    if (u > pairs) u = pairs;
-    return u < 1 ? 1 : u;
+    const int cap = device_units(dev, h_q, s_q);
+    if (cap < 1) return MLA_ERR_CUDA;
+    const int u = units_bound(num_sms, h_q, s_q);
+    return u > cap ? cap : u;
+}
+
+mla_status mla_test_set_stall(int stall, unsigned long long wait_limit_ns) {
+    if (stall != 0 && stall != 1) return MLA_ERR_INVALID_ARG;
+    const unsigned long long limit = wait_limit_ns == 0 ? 2000000000ull : wait_limit_ns;
+    if (cudaMemcpyToSymbol(g_mla_debug_stall, &stall, sizeof(stall)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_mla_wait_limit_ns, &limit, sizeof(limit)) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    return MLA_OK;
 }
 
 mla_status mla_get_metadata(const int32_t* seqlens, int batch, int h_q, int s_q, int num_sms,
                             int32_t* metadata, int32_t* num_splits, void* stream) {
     if (!seqlens || !metadata || !num_splits || num_sms < 1) return MLA_ERR_INVALID_ARG;
     if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
-    const int units = mla_num_work_units(num_sms);
+    const int units = mla_num_work_units(num_sms, h_q, s_q);
     if (units < 0) return units;
     const int tiles = num_tiles(h_q, s_q);
     const size_t table = ((size_t)batch * tiles + 1 + (size_t)batch) * sizeof(int32_t);
@@ -359,10 +465,10 @@ mla_status mla_decode_fwd_simt(const uint16_t* q, const uint16_t* kcache, int nu
                                  workspace, workspace_bytes, out, lse);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-    const int pairs = device_pairs(dev);
-    if (pairs < 1) return MLA_ERR_CUDA;
+    const int units = device_units(dev, h_q, s_q);
+    if (units < 1) return MLA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    decode_simt_kernel<<<2 * pairs, kSimtThreads, 0, s>>>(p);
+    decode_simt_kernel<<<units, kSimtThreads, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return launch_combine(p, s);
 }
@@ -427,26 +533,16 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
                                     batch, s_q, h_q, scale, causal, metadata, num_splits,
                                     scratch, scratch_bytes, out, lse);
     if (st != MLA_OK) return st;
-    const int pairs = device_pairs(dev);
-    if (pairs < 1 || !prepare_split_kernel(dev)) return MLA_ERR_CUDA;
+    const int units = device_units(dev, h_q, s_q);
+    if (units < 1) return MLA_ERR_CUDA;
     // worst case over every schedule this device can run: one chunk per work sequence
     // plus one per unit
-    if (mla_workspace_bytes(batch, h_q, s_q, 2 * pairs) > scratch_bytes)
+    if (workspace_bytes_for((size_t)batch * num_tiles(h_q, s_q) + (size_t)units) > scratch_bytes)
         return MLA_ERR_WORKSPACE_TOO_SMALL;
     DecodeParams p = make_params(q, kcache, num_blocks, block_table, max_blocks, seqlens,
                                  batch, s_q, h_q, scale, causal, metadata, num_splits,
                                  scratch, scratch_bytes, out, lse);
-    CUtensorMap tm_page, tm_pair, tm_q4, tm_q5;
-    const size_t q_rows = (size_t)batch * s_q * h_q;
-    if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
-        !make_page_map(&tm_pair, kcache, num_blocks, 2) ||
-        !make_q_map(&tm_q4, q, q_rows, 4) || !make_q_map(&tm_q5, q, q_rows, 5))
-        return MLA_ERR_CUDA;
-    cudaStream_t s = (cudaStream_t)stream;
-    pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair,
-                                                                          tm_q4, tm_q5);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-    return launch_combine(p, s);
+    return launch_decode(p, q, kcache, num_blocks, (cudaStream_t)stream);
 }
 
 mla_status mla_kv_append(const uint16_t* kv_new, int s_new, const int32_t* block_table,

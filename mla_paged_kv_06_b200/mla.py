@@ -47,7 +47,8 @@ def _load() -> ctypes.CDLL:
         "mla_metadata_ints": (sz, [i32]),
         "mla_num_splits_len": (sz, [i32, i32, i32]),
         "mla_workspace_bytes": (sz, [i32, i32, i32, i32]),
-        "mla_num_work_units": (i32, [i32]),
+        "mla_num_work_units": (i32, [i32, i32, i32]),
+        "mla_test_set_stall": (i32, [i32, ctypes.c_ulonglong]),
         "mla_get_metadata": (i32, [vp, i32, i32, i32, i32, vp, vp, vp]),
         "mla_decode_fwd": (i32, [vp, vp, i32, vp, i32, vp, i32, i32, i32, f32, i32,
                                  vp, vp, vp, sz, vp, vp, vp]),
@@ -117,11 +118,17 @@ def mla_workspace_bytes(batch: int, h_q: int, s_q: int, num_sms: int) -> int:
     return _lib.mla_workspace_bytes(batch, h_q, s_q, num_sms)
 
 
-def mla_num_work_units(num_sms: int) -> int:
-    n = _lib.mla_num_work_units(num_sms)
+def mla_num_work_units(num_sms: int, h_q: int = 128, s_q: int = 1) -> int:
+    n = _lib.mla_num_work_units(num_sms, h_q, s_q)
     if n < 0:
         raise MlaError(n, "mla_num_work_units")
     return n
+
+
+def mla_test_set_stall(stall: bool, wait_limit_ns: int = 0):
+    """Test hook: make every decode kernel launched afterwards stall before its first copy
+    (each wait then gives up after wait_limit_ns); stall=False restores normal decoding."""
+    _check(_lib.mla_test_set_stall(1 if stall else 0, wait_limit_ns), "mla_test_set_stall")
 
 
 def default_num_sms(device=None) -> int:

@@ -1,10 +1,18 @@
 """GPU parity of the CUDA decode path against the fp64 CPU oracle, through the C ABI.
 
 Tolerances (the decode's accuracy contract): max |out - oracle| <= 1e-2 on the bf16
-output and max |lse - oracle| <= 1e-3 on the fp32 log-sum-exp. Small cases compare every
-element; the full-size workloads run in the benchmark's launch configuration (all SMs)
-and compare sampled sequences the oracle computes one by one, plus properties that hold
-at any size (finite outputs, agreement with the no-split schedule).
+output and max |lse - oracle| <= 1e-3 on the fp32 log-sum-exp. Because long sequences
+have small outputs (about 1/sqrt(visible tokens)), an absolute bound alone is loose
+there, so every comparison also bounds the error of each row relative to that row's
+largest output: max_d |out - oracle| / max_d |oracle| <= 2e-2. The derivation: the bf16
+rounding of the output contributes at most 2^-9 = 0.002 of the row maximum; the bf16
+rounding of the probabilities P before the PV product perturbs each term of the weighted
+sum by at most 2^-9 relative, which for an output that sums n comparable terms of
+random sign is about 2^-9 / sqrt(3) = 0.0011 of the row's scale per element (times a
+few standard deviations over 512 dims and up to 128 rows); 2e-2 leaves a factor of
+several over both. Small cases and the full-size workloads (every sequence, in the
+benchmark's launch configuration) compare every element with the oracle; a few
+properties are checked besides (finite outputs, agreement with the no-split schedule).
 """
 
 import numpy as np
@@ -18,6 +26,7 @@ pytestmark = pytest.mark.gpu
 
 ATOL_OUT = 1e-2
 ATOL_LSE = 1e-3
+REL_OUT = 2e-2          # per row: max |dout| / max |out_oracle|
 # Two GPU results that are each within the tolerance of the oracle can differ by twice
 # it (one bf16 ulp is 0.0156 at |o| in [2, 4)), so GPU-vs-GPU comparisons use 2x.
 ATOL_PAIR_OUT = 2 * ATOL_OUT
@@ -59,7 +68,20 @@ def compare(out, lse, ref_out, ref_lse, what=""):
     d_l = np.abs(l[fin] - ref_lse[fin]).max() if fin.any() else 0.0
     assert d_o <= ATOL_OUT, f"{what}: max|dout|={d_o:.3e}"
     assert d_l <= ATOL_LSE, f"{what}: max|dlse|={d_l:.3e}"
-    return d_o, d_l
+    rel = row_relative_error(o, ref_out)
+    assert rel <= REL_OUT, f"{what}: max row-relative error {rel:.3e}"
+    return d_o, d_l, rel
+
+
+def row_relative_error(o, ref_out):
+    """Largest over rows of max_d |o - ref| / max_d |ref| (rows whose reference is all
+    zero, the empty rows, are compared absolutely above and skipped here)."""
+    if o.size == 0:
+        return 0.0
+    err = np.abs(o - ref_out).reshape(-1, ref_out.shape[-1]).max(axis=1)
+    scale = np.abs(ref_out).reshape(-1, ref_out.shape[-1]).max(axis=1)
+    nz = scale > 0
+    return float((err[nz] / scale[nz]).max()) if nz.any() else 0.0
 
 
 def oracle_all(x):
@@ -110,7 +132,7 @@ def test_device_metadata_matches_host_plan():
         seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
         for nsm in [1, 2, 13, mla.default_num_sms()]:
             meta, ns = mla.mla_get_metadata(seq, h_q, s_q, nsm)
-            units = mla.mla_num_work_units(nsm)
+            units = mla.mla_num_work_units(nsm, h_q, s_q)
             hm, hns = mla.mla_plan_host(lens, h_q, s_q, units)
             assert np.array_equal(meta.cpu().numpy()[: hm.size], hm)
             assert np.array_equal(ns.cpu().numpy(), hns)
@@ -120,7 +142,7 @@ def test_more_units_than_clusters():
     # A host-planned schedule with more units than the split kernel has clusters: each
     # cluster then runs several units one after another, and the result is unchanged.
     mla = _mla()
-    units = 3 * mla.mla_num_work_units(mla.default_num_sms()) + 5
+    units = 3 * mla.mla_num_work_units(mla.default_num_sms(), 128, 1) + 5
     lens = [3000, 200, 5000, 64, 1, 0, 777, 4100]
     x = wl.make_paged_inputs(lens, 1, 128, seed=71, spare_blocks=2, poison=True)
     hm, hns = mla.mla_plan_host(lens, 128, 1, units)
@@ -165,15 +187,6 @@ def test_thirty_thousand_sequences_sharing_a_small_pool():
 FULL = ["uniform", "v3", "spec", "skewed"]
 
 
-def _sample(x, k=6):
-    lens = x.seqlens.tolist()
-    order = sorted(range(len(lens)), key=lambda b: lens[b])
-    g = np.random.default_rng(7)
-    pick = {order[0], order[-1], order[len(order) // 2]}
-    pick |= set(g.choice(len(lens), size=min(k, len(lens)), replace=False).tolist())
-    return sorted(pick)
-
-
 @pytest.fixture(scope="module")
 def full_inputs():
     cache = {}
@@ -188,15 +201,14 @@ def full_inputs():
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_workload_sampled_parity(name, full_inputs):
+def test_full_workload_parity(name, full_inputs):
+    # every sequence of the full-size workload, element by element, in the benchmark's
+    # launch configuration (all SMs, the device scheduler's split schedule)
     x, d = full_inputs(name)
     out, lse = run(x, d)
-    o = out.double().cpu().numpy()
-    assert np.isfinite(o).all()
-    idx = _sample(x)
-    ref_out, ref_lse = oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale,
-                                     x.causal, batch_indices=idx)
-    compare(out[idx], lse[idx], ref_out, ref_lse, what=name)
+    ref_out, ref_lse = oracle_all(x)
+    d_o, d_l, rel = compare(out, lse, ref_out, ref_lse, what=name)
+    print(f"{name}: max|dout| {d_o:.3e}  max|dlse| {d_l:.3e}  max row-relative {rel:.3e}")
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -221,10 +233,7 @@ def test_nan_poison_full_size():
     assert torch.isnan(x.kcache[:, :, 0, 0].float()).any()
     out, lse = run(x)
     assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
-    idx = _sample(x, 3)
-    ref = oracle.decode(x.q, x.kcache, x.block_table, x.seqlens, x.scale, x.causal,
-                        batch_indices=idx)
-    compare(out[idx], lse[idx], *ref, what="v3-poison")
+    compare(out, lse, *oracle_all(x), what="v3-poison")
 
 
 @pytest.mark.parametrize("impl", ["tc", "simt"])
@@ -275,3 +284,24 @@ def test_bad_inputs_report_device_error():
     assert st == mla.MLA_ERR_DEVICE_BAD_INPUT
     st, _ = mla.mla_get_last_device_error()
     assert st == mla.MLA_OK
+
+
+@pytest.mark.parametrize("h_q", [16, 128])          # the 1-CTA and the 2-CTA kernel
+def test_bounded_wait_gives_up_and_reports_a_timeout(h_q):
+    # The test hook makes each CTA's loader wait, before its first copy, on a barrier that
+    # nothing completes. Every wait of the kernel then gives up after the (here 2 ms)
+    # limit: the launch ends normally with MLA_ERR_DEVICE_TIMEOUT recorded, nothing is in
+    # flight, and the device stays usable for the next call.
+    mla = _mla()
+    x = wl.make_paged_inputs([300, 70, 1], 1, h_q, seed=31)
+    d = to_dev(x)
+    mla.mla_test_set_stall(True, 2_000_000)
+    try:
+        run(x, d, check_error=False)
+        st, word = mla.mla_get_last_device_error()
+    finally:
+        mla.mla_test_set_stall(False, 0)
+    assert st == mla.MLA_ERR_DEVICE_TIMEOUT, (mla.status_string(st), hex(word))
+    assert word & 0xFF == 1                          # the timeout kind
+    out, lse = run(x, d)
+    compare(out, lse, *oracle_all(x), what="after a timeout")
