@@ -27,14 +27,20 @@ Quantizing a bf16 row, group g = dims [128g, 128g + 128):
     amax_g  = max |x_d| over the group                       (exact)
     s_g     = fp32(amax_g / 448)                             (fp32 division, nearest-even)
     code_d  = E4M3(fp32(x_d / s_g)), nearest-even, saturated to +-448    (0 when s_g = 0)
-The integer codes are decided in fp32, the precision a kernel would use. Dequantizing:
-    x^_d = E4M3 value(code_d) * s_g                          (exact in fp64)
-and rope dims are read back as they were. Decode over an FP8 cache is exact attention
-(the bf16 oracle's definition) over the dequantized rows x^.
+The integer codes are decided in fp32, the precision a kernel would use. Reading back:
+    x^_d = bf16(fp32(E4M3 value(code_d) * s_g))     (fp32 product, then bf16, both
+                                                     round-to-nearest-even)
+and rope dims are read back as they were. The read-back value is a bf16 number: the
+operand type a tensor-core decode multiplies, so a decode kernel widens every page into
+exactly these values and the CPU side takes the same two roundings in the same order.
+Their cost (2^-9 relative at most, with the fp32 step far below it) is small beside the
+format's own 2^-4 step. Decode over an FP8 cache is exact attention (the bf16 oracle's
+definition) over the read-back rows x^.
 
 Pins (tests/test_fp8_oracle.py, no GPU): every code against torch's float8_e4m3fn, the
 encoder against torch's cast on values in range, saturation and rounding ties by the
-definition, the round trip of representable values, the error bound of the format, the
+definition, the read-back against torch's fp32 product and bf16 cast, the bf16 rounding
+on its ties, the round trip of representable values, the error bound of the format, the
 byte layout on a hand-built row, and decode against the brute-force loop on the
 dequantized cache.
 """
@@ -121,12 +127,27 @@ def quantize_rows(rows) -> np.ndarray:
     return out
 
 
+def round_to_bf16(x32) -> np.ndarray:
+    """fp32 values rounded to the nearest bf16 value (ties to even), returned as fp32:
+    on the bit pattern, add 0x7FFF plus the lowest kept bit and drop the low 16 bits.
+    NaN stays NaN; the format's products never reach the overflow range."""
+    x32 = np.asarray(x32, dtype=np.float32)
+    bits = x32.view(np.uint32).astype(np.uint64)
+    lsb = (bits >> 16) & 1
+    r = (((bits + 0x7FFF + lsb) >> 16) << 16).astype(np.uint32).view(np.float32)
+    return np.where(np.isnan(x32), np.float32(np.nan), r)
+
+
 def dequantize_rows(q) -> np.ndarray:
-    """[n, 656] uint8 rows -> [n, 576] fp64 values (latent dims exactly code * scale)."""
+    """[n, 656] uint8 rows -> [n, 576] fp64 values: latent dims bf16(fp32(code * scale)),
+    rope dims as stored."""
     q = np.asarray(q, dtype=np.uint8).reshape(-1, ROW_BYTES)
     n = q.shape[0]
-    scales = q[:, SCALE_OFF:ROPE_OFF].copy().view("<f4").astype(np.float64)
-    lat = e4m3_value(q[:, :LATENT]).reshape(n, GROUPS, GROUP) * scales[:, :, None]
+    scales = q[:, SCALE_OFF:ROPE_OFF].copy().view("<f4")                      # fp32
+    vals = e4m3_value(q[:, :LATENT]).astype(np.float32).reshape(n, GROUPS, GROUP)  # exact
+    with np.errstate(invalid="ignore", over="ignore"):
+        prod = (vals * scales[:, :, None]).astype(np.float32)                   # fp32, nearest-even
+    lat = round_to_bf16(prod).astype(np.float64)
     rope = _bits_to_f32(q[:, ROPE_OFF:].copy().view("<u2")).astype(np.float64)
     return np.concatenate([lat.reshape(n, LATENT), rope], axis=1)
 

@@ -75,9 +75,11 @@ def test_byte_layout_of_a_hand_built_row():
     assert np.array_equal(q[528:656].copy().view("<i2"), rope_bits)
     back = f8.dequantize_rows(q[None])[0]
     assert back[0] == 448.0 and back[1] == -1.0 and back[128] == 3.5     # scales 1 and 2^-7
-    # amax 0.25 comes back as 448 times the fp32-rounded scale 0.25 / 448
-    assert back[384] == -448.0 * float(np.float32(0.25) / np.float32(448.0))
-    assert abs(back[384] + 0.25) <= 0.25 * 2.0 ** -24
+    # amax 0.25 comes back as 448 times the fp32-rounded scale 0.25 / 448, in fp32, then
+    # rounded to bf16: within 2^-24 of 0.25 before the bf16 step, exactly 0.25 after it
+    prod = np.float32(448.0) * (np.float32(0.25) / np.float32(448.0))
+    assert abs(float(prod) - 0.25) <= 0.25 * 2.0 ** -23
+    assert back[384] == -0.25
     assert np.array_equal(back[512:], rope)
 
 
@@ -102,7 +104,9 @@ def test_representable_values_round_trip_exactly():
 
 def test_quantization_error_is_within_the_format_bound():
     # per element: at most half a step of the value's binade (2^-4 relative for normal
-    # values), and at most half the subnormal step (2^-10 * scale) below 2^-6 * scale
+    # values), and at most half the subnormal step (2^-10 * scale) below 2^-6 * scale;
+    # the read-back then adds the fp32 product's and the bf16 rounding (2^-24 + 2^-9 of the
+    # read-back value)
     x = wl.make_paged_inputs([300], 1, 1, seed=2).kcache.reshape(-1, 576)[:300]
     ref = x.float().double().numpy()
     back = f8.dequantize_rows(f8.quantize_rows(x))
@@ -111,9 +115,35 @@ def test_quantization_error_is_within_the_format_bound():
     scales = q[:, 512:528].copy().view("<f4").astype(np.float64)
     s = np.repeat(scales, 128, axis=1)
     err = np.abs(back[:, :512] - ref[:, :512])
-    bound = np.maximum(np.abs(ref[:, :512]) * 2.0 ** -4, s * 2.0 ** -10) * (1 + 1e-6)
+    bound = (np.maximum(np.abs(ref[:, :512]) * 2.0 ** -4, s * 2.0 ** -10) * (1 + 1e-6)
+             + np.abs(back[:, :512]) * (2.0 ** -9 + 2.0 ** -24))
     assert np.all(err <= bound)
     assert err.max() > 0                                # it is a lossy format
+
+
+def test_read_back_is_the_fp32_product_rounded_to_bf16():
+    # an independent route to the same value: torch's E4M3 decode, an fp32 multiply and
+    # torch's round-to-nearest-even cast to bf16
+    x = wl.make_paged_inputs([200], 1, 1, seed=6).kcache.reshape(-1, 576)[:200]
+    q = f8.quantize_rows(x)
+    codes = torch.from_numpy(q[:, :512].copy()).view(torch.float8_e4m3fn).float()
+    scales = torch.from_numpy(q[:, 512:528].copy().view("<f4")).repeat_interleave(128, dim=1)
+    want = (codes * scales).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(f8.dequantize_rows(q)[:, :512], want)
+
+
+def test_bf16_rounding_ties_and_specials():
+    # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: ties go to the even mantissa (1);
+    # 1 + 3 * 2^-8 halfway between 1 + 2^-7 and 1 + 2^-6: to 1 + 2^-6; just above a tie
+    # rounds up; NaN stays NaN
+    x = np.float32([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 1 + 2.0 ** -8 + 2.0 ** -20, -2.5, np.nan])
+    r = f8.round_to_bf16(x)
+    assert r[0] == 1.0 and r[1] == 1 + 2.0 ** -6 and r[2] == 1 + 2.0 ** -7 and r[3] == -2.5
+    assert np.isnan(r[4])
+    g = np.random.default_rng(7)
+    y = (g.standard_normal(200_000) * np.exp(g.uniform(-30, 30, 200_000))).astype(np.float32)
+    want = torch.from_numpy(y).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(f8.round_to_bf16(y), want)
 
 
 def test_fp8_decode_matches_brute_force_on_the_dequantized_cache():
