@@ -364,6 +364,65 @@ def time_config(mla, name, seed, flush, stream, steps, warmup, hbm_peak, tf_peak
     return entry
 
 
+def time_fp8(mla, seed, flush, stream, steps, warmup, hbm_peak):
+    """Decode over an FP8 latent cache (mla_decode_fwd_fp8) on the uniform workload's
+    shape, timed like the main measurement. The cache is the uniform pool quantized on the
+    GPU by mla_kv_append_fp8 (16 rows per page per call); algorithmic bytes count 656 per
+    token (the row format) plus q, out and lse."""
+    x = wl.make_workload("uniform", seed=seed)
+    nb = x.num_blocks
+    kc8 = torch.zeros((nb, 64, mla.MLA_FP8_ROW_BYTES), dtype=torch.uint8, device="cuda")
+    rows = x.kcache.view(nb, 64, 576).cuda()
+    ident = torch.arange(nb, dtype=torch.int32, device="cuda").view(nb, 1)
+    for j in range(4):
+        at = torch.full((nb,), 16 * j, dtype=torch.int32, device="cuda")
+        mla.mla_kv_append_fp8(rows[:, 16 * j:16 * (j + 1)].contiguous(), ident, at, kc8)
+    del rows
+    d = dict(q=x.q.cuda(), block_table=x.block_table.cuda(), seqlens=x.seqlens.cuda())
+    nsm = mla.default_num_sms()
+    meta = torch.empty(mla.mla_metadata_ints(nsm), dtype=torch.int32, device="cuda")
+    ns = torch.empty(mla.mla_num_splits_len(x.batch, x.h_q, x.s_q), dtype=torch.int32,
+                     device="cuda")
+    ws = torch.empty(mla.mla_workspace_bytes(x.batch, x.h_q, x.s_q, nsm), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((x.batch, x.s_q, x.h_q, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
+
+    def call():
+        mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
+        mla.mla_decode_fwd_fp8(d["q"], kc8, d["block_table"], d["seqlens"], x.scale, x.causal,
+                               meta, ns, ws, out, lse)
+
+    for _ in range(max(warmup, 3)):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    st, word = mla.mla_get_last_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the FP8 decode: {mla.status_string(st)} {word:#x}")
+    tokens = int(x.seqlens.sum())
+    rows_total = x.batch * x.s_q * x.h_q
+    nbytes = tokens * mla.MLA_FP8_ROW_BYTES + rows_total * (1152 + 1024 + 4)
+    us = statistics.median(ts)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"workload": "uniform shape over an FP8 cache (656-byte rows: E4M3 latent codes, "
+                        "four fp32 group scales, bf16 rope)",
+            "us_per_call": us, "GB/s": gbs, "hbm_frac": gbs / hbm_peak,
+            "algorithmic_bytes": nbytes,
+            "bf16_cache_bytes_same_workload": tokens * 1152 + rows_total * (1152 + 1024 + 4),
+            "note": "metadata + mla_decode_fwd_fp8 per call, L2 flushed before each; the "
+                    "cache was quantized on the GPU by mla_kv_append_fp8"}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -548,6 +607,8 @@ def main():
     split_kv = time_split_kv(mla, flush, stream, args.steps, args.seed) if args.split_kv > 1 else None
 
     hbm_peak, tf_peak, peak_kind = peaks()
+    fp8 = None if args.no_configs else time_fp8(mla, rank_seed(args.seed, rank), flush, stream,
+                                                args.steps, args.warmup, hbm_peak)
     # every workload of the benchmark in the same run, each against its own roofline
     configs = {}
     if not args.no_configs:
@@ -618,6 +679,7 @@ def main():
                               "note": "mla_kv_append_fp8: the same rows quantized into the "
                                       "656-byte FP8 row format, replayed from a CUDA graph"},
             "split_kv": split_kv,
+            "fp8_cache": fp8,
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x, args.cpu_seconds)

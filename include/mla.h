@@ -116,7 +116,9 @@ int mla_num_work_units(int num_sms, int h_q, int s_q);
  *   num_sms     SMs the decode may use (>= 1); 148 on a B200. num_sms = 1 forces a
  *               single unit and so no splits.
  *   metadata    device int32 [mla_metadata_ints(num_sms)], written:
- *               [0..7]   header {num_units, tiles, batch, h_q, s_q, unit_cost, 0, 0}
+ *               [0..7]   header {num_units, tiles, batch, h_q, s_q, unit_cost,
+ *                        item_overhead, 0}: a work sequence costs its pages plus
+ *                        item_overhead (3 for the 2-CTA kernel, 1 for the 1-CTA kernel)
  *               [8u+8..] unit u {v_begin, page_begin, v_end, page_end, chunk_begin,0,0,0}
  *                        (half-open range of (v, page) positions)
  *   num_splits  device int32 [mla_num_splits_len(batch, h_q, s_q)], written: the
@@ -278,12 +280,39 @@ mla_status mla_kv_append(const uint16_t* kv_new, int s_new, const int32_t* block
  * Supported: 1 <= s_new <= 16, 1 <= batch <= 65536. Invalid arguments return an error
  * before any launch; a position past the block table or a block id outside the pool is a
  * device-side bad input and that row is not written. A group holding a NaN gets NaN codes
- * and a NaN scale. Asynchronous on `stream`; allocates nothing. (A decode over this
- * format is not provided yet.)
+ * and a NaN scale. Asynchronous on `stream`; allocates nothing. mla_decode_fwd_fp8
+ * decodes over this format.
  */
 mla_status mla_kv_append_fp8(const uint16_t* kv_new, int s_new, const int32_t* block_table,
                              int max_blocks, const int32_t* seqlens, int batch,
                              uint8_t* kcache_fp8, int num_blocks, void* stream);
+
+/*
+ * Decode attention over an FP8 latent cache in the row format of mla_kv_append_fp8:
+ * exactly mla_decode_fwd's operation over the rows as the format reads them back,
+ *     latent dim d of group g:  bf16(fp32(E4M3 value(code_d) * s_g))   (both nearest-even)
+ *     rope dims:                as stored (bf16)
+ * so its results are those of mla_decode_fwd over a bf16 cache holding the read-back
+ * rows, within the same tolerances. The format is this library's (the pages use FP8 for
+ * GEMMs with fine-grained scale factors, the DeepGEMM page's paragraph on fine-grained
+ * scaling, not for the KV cache). It streams 656 bytes per token instead of 1,152.
+ *
+ *   kcache_fp8  device uint8 [num_blocks][64][656] (MLA_FP8_ROW_BYTES per row),
+ *               16-byte aligned (read)
+ *   every other argument as for mla_decode_fwd, with metadata, num_splits and the
+ *   workspace size from the same calls for the same shapes.
+ * Supported: s_q * h_q <= 32 (the kernel's two 33 KB staging buffers fit beside its
+ * bf16 stages only for up to 32 query rows); larger row counts return
+ * MLA_ERR_UNSUPPORTED before any launch. The 1-CTA kernel widens each page into bf16 in
+ * shared memory before its QK; codes of rows past a sequence's end are never read.
+ */
+mla_status mla_decode_fwd_fp8(const uint16_t* q, const uint8_t* kcache_fp8, int num_blocks,
+                              const int32_t* block_table, int max_blocks,
+                              const int32_t* seqlens, int batch, int s_q, int h_q,
+                              float scale, int causal,
+                              const int32_t* metadata, const int32_t* num_splits,
+                              void* workspace, size_t workspace_bytes,
+                              uint16_t* out, float* lse, void* stream);
 
 /*
  * Reads and clears the device-side error word of the current device after

@@ -5,30 +5,39 @@
 // rows or fewer, one of its CTAs computes padding only, yet the pair still runs its full
 // per-page chain, including the post-QK reload of the other page. Here one CTA owns a
 // work unit alone and reads every page exactly once:
-//   QK:  S = Q K^T for one 64-token page: M = 128 (the R <= 64 real query rows; the rows
-//        beyond are never read), N = 64 tokens, K = 576. Q's first kQtChunks x 64 dims
-//        come from TMEM, the rest from shared memory. S lands one query row per TMEM
-//        lane, so one thread owns a whole row: the row max needs no exchange.
+//   QK:  S = Q K^T for one 64-token page: M = 128, N = 64 tokens, K = 576. The A operand
+//        holds the R <= 64 query rows replicated: TMEM lane l (A row l) carries query row
+//        l % 32 (kN <= 32: four copies, one per lane quarter) or l % 64 (kN = 64: two
+//        copies). So every warp finds every row's scores in its own lane quarter, and
+//        the four warps split each page's tokens between them: the softmax work of a
+//        page is spread over all four SM sub-partitions instead of one or two.
+//        Q's first kQtChunks x 64 dims come from TMEM, the rest from shared memory (the
+//        replicated rows laid out as 128 A rows).
 //   PV:  transposed, O^T = V^T P^T: M = 128 latent dims (four blocks for 512), N = kN
 //        (the rows padded to 16, 32 or 64), K = 16 tokens per instruction. V^T is the page
 //        tile itself, read MN-major from its stage (no copy); P is the B operand, K-major,
-//        one 128-byte row of 64 bf16 probabilities per query row. O^T needs 4 kN TMEM
-//        columns, which leaves room for Q in TMEM and two score buffers.
+//        one 128-byte row of 64 bf16 probabilities per query row, each warp writing its
+//        token slice. O^T needs 4 kN TMEM columns, which leaves room for Q in TMEM.
 // Per CTA (192 threads):
-//   warps 0-3  the row group. Thread r (TMEM lane r) does the softmax of query row r < R.
-//              All 128 threads (TMEM lane = latent dim of an O^T block) do the rare O
-//              rescale, the epilogue, the move of each item's q rows into TMEM and shared
-//              memory, and the zeroing of V rows past a sequence's end.
+//   warps 0-3  the row group. Warp w takes copy w / kRowWarps of the rows (token slice
+//              [copy x kTok, +kTok) of every page) and rows (w % kRowWarps) x 32 + lane.
+//              All 128 threads (TMEM lane = latent dim of an O^T block) also do the rare
+//              O rescale, the epilogue, the move of each item's q rows into TMEM and
+//              shared memory, and the zeroing of V rows past a sequence's end.
 //   warp 4     TMA producer: a ring of kStages 72 KB stages. An item takes one slot for its
 //              q rows (box {64, kN rows, 9 chunks}) and then one slot per page (box {64,
 //              64 rows, 9 chunks}: 9 swizzled 8 KB tiles in one instruction), with the next
 //              page prefetched into L2.
-//   warp 5     TMEM owner and MMA issuer. Issue order QK(j), QK(j+1), PV(j), QK(j+2), ...
-//              keeps the tensor pipe busy while the row group computes P(j).
+//   warp 5     TMEM owner and MMA issuer, in the order QK(0) QK(1) PV(0) QK(2) PV(1) ...:
+//              the next page's QK keeps the tensor pipe busy while the row group turns
+//              S(j) into P(j).
 // Scores stay in the log2 domain. A row's reference max is raised only when a score
-// exceeds it by more than kRescaleLog2; O^T columns are then rescaled in TMEM by all four
-// warps (a column spans all 128 lanes).
+// exceeds it by more than kRescaleLog2. Partial maxima of the token slices meet in shared
+// memory once per page; every warp then tracks every row's reference itself, so the
+// rescale factors of O^T columns need no second exchange.
 #pragma once
+
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "items.cuh"
@@ -47,27 +56,42 @@ constexpr uint32_t kStageBytes = 9 * kBoxBytes;      // one page: 64 tokens x 57
 constexpr uint32_t kSmemLimit = 232448;              // sm_100 per-block opt-in maximum
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxStages = 3;
+constexpr int kQkChunk = 9;                          // K-steps of QK per issue burst
 
-// Layout for kN padded query rows. TMEM columns: O^T [0, 4 kN), two score buffers of 64,
+// Layout for kN padded query rows. TMEM columns: O^T [0, 4 kN), kSBufs score buffers of 64,
 // then Q's first dims as bf16 pairs. Shared memory (from a 1 KB aligned base): Q's
-// remaining chunks, one P buffer, the stages, then barriers and per-row arrays.
-template <int N_>
+// remaining chunks (128 replicated A rows each), one P buffer, the stages, then barriers
+// and per-row arrays.
+template <int N_, bool F8_ = false>
 struct Cfg {
     static constexpr int kN = N_;
+    static constexpr bool kF8 = F8_;                          // FP8 latent cache (656-byte rows)
+    static constexpr int kRowWarps = kN <= 32 ? 1 : 2;        // warps holding one copy of the rows
+    static constexpr int kCopies = 4 / kRowWarps;
+    static constexpr int kTok = 64 / kCopies;                 // tokens of a page per warp
     static constexpr uint32_t kColO = 0;
     static constexpr uint32_t kColS = 4 * kN;
-    static constexpr uint32_t kColQ = kColS + 128;
+    static constexpr int kSBufs = (kColS + 2 * 64 + 288 <= kTmemCols) ? 2 : 1;
+    static constexpr uint32_t kColQ = kColS + 64 * kSBufs;
     static constexpr int kQtChunksFit = (int)((kTmemCols - kColQ) * 2 / 64);
     static constexpr int kQtChunks = kQtChunksFit >= 9 ? 9 : kQtChunksFit;   // Q chunks in TMEM
     static constexpr int kQsChunks = 9 - kQtChunks;                          // in shared memory
     static constexpr uint32_t kTileBytes = kN * 128;          // kN rows x 64 dims, one chunk
+    static constexpr uint32_t kARows = 128;                   // A rows of a Q chunk in smem
     static constexpr uint32_t kOffQs = 0;
-    static constexpr uint32_t kOffP = kOffQs + kQsChunks * kTileBytes;
+    static constexpr uint32_t kOffP = kOffQs + kQsChunks * kARows * 128;
     static constexpr uint32_t kOffStage = kOffP + kTileBytes;
-    static constexpr uint32_t kMiscBytes = 1024;
-    static constexpr int kStagesFit = (int)((kSmemLimit - 1024 - kMiscBytes - kOffStage) / kStageBytes);
-    static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
-    static constexpr uint32_t kOffMisc = kOffStage + kStages * kStageBytes;
+    static constexpr uint32_t kMiscBytes = 4096;
+    // FP8 cache: a page's codes and scales (64 rows x 528 bytes) land in one of two staging
+    // buffers and are widened into a bf16 stage; the rope dims land in the stage directly
+    static constexpr uint32_t kF8RowBytes = 528;
+    static constexpr uint32_t kF8PageBytes = 64 * kF8RowBytes;          // 33,792 (33 KB)
+    static constexpr int kF8Stages = kF8 ? 2 : 0;
+    static constexpr int kStagesFit =
+        (int)((kSmemLimit - 1024 - kMiscBytes - kOffStage - kF8Stages * kF8PageBytes) / kStageBytes);
+    static constexpr int kStages = kF8 ? 2 : (kStagesFit > kMaxStages ? kMaxStages : kStagesFit);
+    static constexpr uint32_t kOffF8 = kOffStage + kStages * kStageBytes;
+    static constexpr uint32_t kOffMisc = kOffF8 + kF8Stages * kF8PageBytes;
     static constexpr uint32_t kSmemAlloc = kOffMisc + kMiscBytes + 1024;     // + base alignment
     static constexpr uint32_t kQSlotBytes = kN * 9 * 128;                    // the q rows' box
     static_assert(kN == 16 || kN == 32 || kN == 64, "kN must be 16, 32 or 64");
@@ -79,46 +103,52 @@ struct Cfg {
 enum : uint32_t {
     kBarFull = 0,                        // [kMaxStages] a stage's copy landed
     kBarFree = kBarFull + kMaxStages,    // [kMaxStages] a stage may be refilled
-    kBarQkDone = kBarFree + kMaxStages,  // [2] QK of a step done (score buffer step % 2)
+    kBarQkDone = kBarFree + kMaxStages,  // [2] QK of a step done (score buffer step % kSBufs)
     kBarPvDone = kBarQkDone + 2,         // PV of a step done (one phase per step)
     kBarPReady = kBarPvDone + 1,         // the row group wrote P (4 warp arrivals)
-    kBarQReady = kBarPReady + 1,         // the item's q rows are in TMEM and shared memory
+    kBarSFree = kBarPReady + 1,          // the row group read S out (single buffer only)
+    kBarQReady = kBarSFree + 1,          // the item's q rows are in TMEM and shared memory
     kBarOFree = kBarQReady + 1,          // the previous item's O^T was read out
-    kBarDecide = kBarOFree + 1,          // the step's rescale decision is posted
-    kBarEpi = kBarDecide + 1,            // the item's row sums are posted
+    kBarDecide = kBarOFree + 1,          // the step's partial maxima are posted
+    kBarEpi = kBarDecide + 1,            // the item's partial row sums / 1/l posted (2 per item)
     kBarDrain = kBarEpi + 1,             // the MMA issuer's last commit
     kBarStall = kBarDrain + 1,           // never completes (the timeout test hook waits on it)
-    kNumBars = kBarStall + 1
+    kBarF8Full = kBarStall + 1,          // [2] FP8 cache: a staging buffer's copy landed
+    kBarF8Free = kBarF8Full + 2,         // [2] FP8 cache: a staging buffer was widened (4 warps)
+    kBarDqFull = kBarF8Free + 2,         // [kMaxStages] FP8 cache: a stage's page widened (4 warps)
+    kNumBars = kBarDqFull + kMaxStages
 };
-// misc area: barriers [0, 128), tmem base at 128, abort flag at 132, rescale tags at 136
-// and 140, rescale factors [2][64] at 256, inverse row sums [64] at 768
-static_assert(kNumBars * 8 <= 128, "barrier area");
+// misc area: barriers [0, 256), tmem base at 256, abort flag at 260; partial maxima
+// [2 parity][4 copies][64 rows] f32 at 512; partial row sums [2 sums][4 copies][64] at
+// 2560; inverse row sums [64] at 3584
+static_assert(kNumBars * 8 <= 256, "barrier area");
+constexpr uint32_t kMiscPmax = 512, kMiscPsum = 2560, kMiscInvL = 3584;
 
-template <int kN>
+template <class C>
 struct Smem {
-    using C = Cfg<kN>;
     uint8_t* base;
     uint32_t base_u32;
     uint64_t wait_limit;                 // ns a wait may last before the kernel gives up
     __device__ uint32_t bar(uint32_t i) const { return base_u32 + C::kOffMisc + 8 * i; }
     __device__ uint32_t stage(uint32_t s) const { return base_u32 + C::kOffStage + s * kStageBytes; }
-    __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + C::kOffMisc + 128); }
+    __device__ uint32_t f8buf(uint32_t f) const { return base_u32 + C::kOffF8 + f * C::kF8PageBytes; }
+    __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + C::kOffMisc + 256); }
     __device__ volatile int* abort_flag() const {
-        return reinterpret_cast<volatile int*>(base + C::kOffMisc + 132);
+        return reinterpret_cast<volatile int*>(base + C::kOffMisc + 260);
     }
-    __device__ volatile int* resc_tag(uint32_t par) const {
-        return reinterpret_cast<volatile int*>(base + C::kOffMisc + 136 + 4 * par);
+    __device__ float* pmax(uint32_t par, int copy) const {
+        return reinterpret_cast<float*>(base + C::kOffMisc + kMiscPmax) + (par * 4 + copy) * 64;
     }
-    __device__ float* facs(uint32_t par) const {
-        return reinterpret_cast<float*>(base + C::kOffMisc + 256 + 256 * par);
+    __device__ float* psum(int which, int copy) const {
+        return reinterpret_cast<float*>(base + C::kOffMisc + kMiscPsum) + (which * 4 + copy) * 64;
     }
-    __device__ float* inv_l() const { return reinterpret_cast<float*>(base + C::kOffMisc + 768); }
+    __device__ float* inv_l() const { return reinterpret_cast<float*>(base + C::kOffMisc + kMiscInvL); }
 };
 
 // Bounded wait: false if the phase does not complete within the limit or another role of
 // the CTA already gave up (then the caller stops).
-template <int kN>
-__device__ __forceinline__ bool wait_bar(const Smem<kN>& sh, uint32_t bar, uint32_t parity,
+template <class C>
+__device__ __forceinline__ bool wait_bar(const Smem<C>& sh, uint32_t bar, uint32_t parity,
                                          uint32_t where) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer();
@@ -136,8 +166,8 @@ __device__ __forceinline__ bool wait_bar(const Smem<kN>& sh, uint32_t bar, uint3
 }
 
 // Warp-uniform bounded wait: no lane leaves while its neighbours stay in .aligned code.
-template <int kN>
-__device__ __forceinline__ bool warp_wait_bar(const Smem<kN>& sh, uint32_t bar, uint32_t parity,
+template <class C>
+__device__ __forceinline__ bool warp_wait_bar(const Smem<C>& sh, uint32_t bar, uint32_t parity,
                                               uint32_t where) {
     const bool ok = wait_bar(sh, bar, parity, where);
     return __all_sync(0xffffffffu, ok);
@@ -146,8 +176,8 @@ __device__ __forceinline__ bool warp_wait_bar(const Smem<kN>& sh, uint32_t bar, 
 // Wait for copies or MMAs this CTA issued before it may finish: bounded by the time limit
 // only (the abort flag does not cut it short, so nothing lands after the CTA has exited
 // unless the limit itself runs out).
-template <int kN>
-__device__ __forceinline__ void drain_wait(const Smem<kN>& sh, uint32_t bar, uint32_t parity,
+template <class C>
+__device__ __forceinline__ void drain_wait(const Smem<C>& sh, uint32_t bar, uint32_t parity,
                                            uint32_t where) {
     const uint64_t t0 = ptx::globaltimer();
     while (!ptx::mbar_try_wait(bar, parity)) {
@@ -165,10 +195,10 @@ __device__ __forceinline__ void warp_arrive(uint32_t bar) {
 
 // ------------------------------------------------------------------ producer (warp 4)
 // Ring slot g uses stage g % kStages; its fill number g / kStages sets the parities.
-template <int kN>
-__device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<kN>& sh,
+template <class C>
+__device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<C>& sh,
                                              const CUtensorMap* tm_page, const CUtensorMap* tm_q) {
-    using C = Cfg<kN>;
+    constexpr int kN = C::kN;
     if (g_mla_debug_stall) {
         // test hook: wait on a barrier nothing completes, before any copy is issued, so
         // every role gives up after the limit with nothing in flight
@@ -211,35 +241,116 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<k
         drain_wait(sh, sh.bar(kBarFull + gg % C::kStages), (gg / C::kStages) & 1u, 0x42u);
 }
 
+// FP8 cache: two cursors over the same items. Cursor A streams each page's codes and
+// scales (box {16 bytes, 33 units, 64 rows}: 528 bytes per row) into the two staging
+// buffers, as far ahead as they free; cursor B fills the bf16 ring in slot order: each
+// item's q rows, then per page its rope dims (box {64, 64 rows} of the bf16 view of the
+// rows, 128-byte swizzle) straight into the stage's rope tile.
+template <class C>
+__device__ __forceinline__ void run_producer_f8(const DecodeParams& p, const Smem<C>& sh,
+                                                const CUtensorMap* tm_codes, const CUtensorMap* tm_rope,
+                                                const CUtensorMap* tm_q) {
+    if (g_mla_debug_stall) {
+        wait_bar(sh, sh.bar(kBarStall), 0, 0x40u);
+        return;
+    }
+    ItemIter ia(p, (int)blockIdx.x, (int)gridDim.x), ib(p, (int)blockIdx.x, (int)gridDim.x);
+    Item a, b;
+    bool have_a = ia.next(a), have_b = ib.next(b);
+    int ka = have_a ? a.k_lo : 0;          // next page of cursor A
+    int kb = -1;                           // next of cursor B: -1 the q slot, else a page
+    uint32_t fa = 0, g = 0;                // staging fills and ring slots issued
+    uint64_t t0 = 0;
+    uint32_t idle = 0;
+    for (;;) {
+        const bool a_ready = have_a && (fa < (uint32_t)C::kF8Stages ||
+            ptx::mbar_test_wait(sh.bar(kBarF8Free + fa % C::kF8Stages), ((fa / C::kF8Stages) - 1u) & 1u));
+        const bool b_ready = have_b && (g < (uint32_t)C::kStages ||
+            ptx::mbar_test_wait(sh.bar(kBarFree + g % C::kStages), ((g / C::kStages) - 1u) & 1u));
+        if (a_ready) {
+            const uint32_t f = fa % C::kF8Stages;
+            ptx::mbar_arrive_expect_tx(sh.bar(kBarF8Full + f), C::kF8PageBytes);
+            ptx::tma_load_3d(sh.f8buf(f), tm_codes, sh.bar(kBarF8Full + f), 0, 0,
+                             page_row(p, a.b, ka, a.k_hi));
+            ++fa;
+            if (++ka >= a.k_hi) { have_a = ia.next(a); ka = have_a ? a.k_lo : 0; }
+            idle = 0;
+        } else if (b_ready) {
+            const uint32_t st = g % C::kStages;
+            if (kb < 0) {
+                ptx::mbar_arrive_expect_tx(sh.bar(kBarFull + st), C::kQSlotBytes);
+                ptx::tma_load_3d(sh.stage(st), tm_q, sh.bar(kBarFull + st), 0,
+                                 b.b * p.rows + b.t * kTileRows, 0);
+                kb = b.k_lo;
+            } else {
+                ptx::mbar_arrive_expect_tx(sh.bar(kBarFull + st), kBoxBytes);
+                ptx::tma_load_2d(sh.stage(st) + 8 * kBoxBytes, tm_rope, sh.bar(kBarFull + st), 0,
+                                 page_row(p, b.b, kb, b.k_hi));
+                if (++kb >= b.k_hi) { have_b = ib.next(b); kb = -1; }
+            }
+            ++g;
+            idle = 0;
+        } else if (!have_a && !have_b) {
+            break;
+        } else if ((++idle & 1023u) == 0) {
+            if (*sh.abort_flag()) break;
+            const uint64_t now = ptx::globaltimer();
+            if (idle == 1024u) t0 = now;
+            else if (now - t0 > sh.wait_limit) {
+                *sh.abort_flag() = 1;
+                record_error(kErrTimeout, 0x43u);
+                break;
+            }
+        }
+    }
+    // every copy issued must land before the CTA may finish
+    for (uint32_t ff = fa > (uint32_t)C::kF8Stages ? fa - C::kF8Stages : 0u; ff < fa; ++ff)
+        drain_wait(sh, sh.bar(kBarF8Full + ff % C::kF8Stages), (ff / C::kF8Stages) & 1u, 0x44u);
+    for (uint32_t gg = g > (uint32_t)C::kStages ? g - C::kStages : 0u; gg < g; ++gg)
+        drain_wait(sh, sh.bar(kBarFull + gg % C::kStages), (gg / C::kStages) & 1u, 0x42u);
+}
+
 // ------------------------------------------------------------------ MMA issuer (warp 5)
-// QK of the page in stage s into score buffer sb, K-steps [k0, k1) of the 36 (16 dims
-// each); the half that ends at 36 commits the buffer's QkDone.
-template <int kN, int k0, int k1>
-__device__ __forceinline__ void issue_qk(const Smem<kN>& sh, uint32_t tmem, uint32_t s, uint32_t sb) {
-    using C = Cfg<kN>;
+// K-steps [k0, k0 + kQkChunk) of the 36 (16 dims each) of QK for the page in stage s into
+// score buffer sb; the last chunk commits the buffer's QkDone.
+template <class C, int k0>
+__device__ __forceinline__ void issue_qk_chunk(const Smem<C>& sh, uint32_t tmem, uint32_t s, uint32_t sb) {
+    constexpr int kN = C::kN;
     constexpr uint32_t kIdesc = ptx::idesc_bf16(128, 64, false, false);
     ptx::tc_fence_after();
     const uint32_t d = tmem + C::kColS + 64 * sb;
     const uint32_t st = sh.stage(s);
 #pragma unroll
-    for (int k = k0; k < k1; ++k) {
+    for (int k = k0; k < k0 + kQkChunk; ++k) {
         const uint64_t bdesc = ptx::smem_desc(st + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024, 2);
         if (k < 4 * C::kQtChunks) {
             ptx::mma_ts(d, tmem + C::kColQ + 8 * k, bdesc, kIdesc, k > 0 ? 1u : 0u);
         } else {
             const uint64_t adesc = ptx::smem_desc(
-                sh.base_u32 + C::kOffQs + ((k >> 2) - C::kQtChunks) * C::kTileBytes + (k & 3) * 32,
+                sh.base_u32 + C::kOffQs + ((k >> 2) - C::kQtChunks) * (C::kARows * 128) + (k & 3) * 32,
                 16, 1024, 2);
             ptx::mma_ss(d, adesc, bdesc, kIdesc, k > 0 ? 1u : 0u);
         }
     }
-    if constexpr (k1 == 36) ptx::mma_commit(sh.bar(kBarQkDone + sb));
+    if constexpr (k0 + kQkChunk == 36) ptx::mma_commit(sh.bar(kBarQkDone + sb));
+}
+
+template <class C>
+__device__ __forceinline__ void issue_qk_chunk(const Smem<C>& sh, uint32_t tmem, uint32_t s,
+                                               uint32_t sb, uint32_t chunk) {
+    static_assert(4 * kQkChunk == 36, "four chunks per QK");
+    switch (chunk) {
+        case 0: issue_qk_chunk<C, 0>(sh, tmem, s, sb); break;
+        case 1: issue_qk_chunk<C, kQkChunk>(sh, tmem, s, sb); break;
+        case 2: issue_qk_chunk<C, 2 * kQkChunk>(sh, tmem, s, sb); break;
+        default: issue_qk_chunk<C, 3 * kQkChunk>(sh, tmem, s, sb); break;
+    }
 }
 
 // O^T += V^T P^T for the page in stage s; `first` starts the item's accumulation.
-template <int kN>
-__device__ __forceinline__ void issue_pv(const Smem<kN>& sh, uint32_t tmem, uint32_t s, bool first) {
-    using C = Cfg<kN>;
+template <class C>
+__device__ __forceinline__ void issue_pv(const Smem<C>& sh, uint32_t tmem, uint32_t s, bool first) {
+    constexpr int kN = C::kN;
     constexpr uint32_t kIdesc = ptx::idesc_bf16(128, kN, true, false);
     ptx::tc_fence_after();
     const uint32_t st = sh.stage(s);
@@ -259,12 +370,13 @@ __device__ __forceinline__ void issue_pv(const Smem<kN>& sh, uint32_t tmem, uint
     ptx::mma_commit(sh.bar(kBarPvDone));
 }
 
-template <int kN>
-__device__ __forceinline__ void run_mma(const DecodeParams& p, const Smem<kN>& sh, uint32_t tmem) {
-    using C = Cfg<kN>;
+template <class C>
+__device__ __forceinline__ void run_mma(const DecodeParams& p, const Smem<C>& sh, uint32_t tmem) {
+    constexpr int kN = C::kN;
     ItemIter iter(p, (int)blockIdx.x, (int)gridDim.x);
     Item it;
     uint32_t g = 0, gs = 0, items = 0;
+    uint32_t dq_par = 0;                   // FP8: bit s = parity of stage s's next widened page
     bool ok = true;
     while (ok && iter.next(it)) {
         // the item's q rows were moved out of their slot: free it
@@ -273,9 +385,7 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Smem<kN>& s
         ptx::mbar_arrive(sh.bar(kBarFree + g % C::kStages));
         ++g;
         const uint32_t n = (uint32_t)it.pages();
-        // Tensor-pipe order QK(0) QK(1) PV(0) QK(2) PV(1) ...: the next page's QK keeps the
-        // pipe busy while the row group turns S(j) into P(j).
-        uint32_t qk = 0, pv = 0;
+        uint32_t qk = 0, kc = 0, pv = 0;   // QKs and PVs issued (kc: chunks of a started QK)
         bool o_free = items == 0;          // the previous item's O^T must be read out first
         uint64_t t0 = 0;
         uint32_t idle = 0;
@@ -284,15 +394,34 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Smem<kN>& s
                 ptx::tc_fence_after();
                 o_free = true;
             }
-            const uint32_t gq = g + qk;
+            const uint32_t gq = g + qk, Sq = gs + qk;
+            bool can_qk = false;
+            if (qk < n) {
+                if (kc > 0) {
+                    can_qk = true;                         // continue the QK in progress
+                } else {
+                    // its score buffer must be free: S of step Sq - kSBufs read out
+                    bool sfree;
+                    if constexpr (C::kSBufs == 2) sfree = qk < pv + 2;
+                    else sfree = Sq == 0 || ptx::mbar_test_wait(sh.bar(kBarSFree), (Sq - 1) & 1u);
+                    const uint32_t st = gq % C::kStages;
+                    can_qk = sfree && ptx::mbar_test_wait(sh.bar(kBarFull + st), (gq / C::kStages) & 1u);
+                    if constexpr (C::kF8)
+                        can_qk = can_qk && ptx::mbar_test_wait(sh.bar(kBarDqFull + st), (dq_par >> st) & 1u);
+                }
+            }
             if (pv < qk && (pv > 0 || o_free) &&
                 ptx::mbar_test_wait(sh.bar(kBarPReady), (gs + pv) & 1u)) {
                 issue_pv(sh, tmem, (g + pv) % C::kStages, pv == 0);
                 ++pv;
                 idle = 0;
-            } else if (qk < n && qk < pv + 2 &&
-                       ptx::mbar_test_wait(sh.bar(kBarFull + gq % C::kStages), (gq / C::kStages) & 1u)) {
-                issue_qk<kN, 0, 36>(sh, tmem, gq % C::kStages, (gs + qk) & 1u);
+            } else if (can_qk) {
+                // a whole QK at once: slipping PVs in between its chunks was measured to
+                // slow the tensor pipe far more than it freed stages early
+                for (uint32_t ck = kc; ck < 4; ++ck)
+                    issue_qk_chunk(sh, tmem, gq % C::kStages, Sq % C::kSBufs, ck);
+                if constexpr (C::kF8) dq_par ^= 1u << (gq % C::kStages);
+                kc = 0;
                 ++qk;
                 idle = 0;
             } else if ((++idle & 1023u) == 0) {
@@ -326,126 +455,218 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* v) {
     else ptx::tmem_ld64(taddr, v);
 }
 
+template <class C>
 struct RowCtx {
     uint32_t tmem, lane_base;
     int tid, warp, lane;
-    bool row_warp;        // the warp holds query rows (warp-uniform)
+    int copy;             // which copy of the rows this warp holds: token slice copy x kTok
+    int row;              // this thread's query row: (warp % kRowWarps) x 32 + lane
+    int own;              // index of `row` among the rows this thread tracks (warp % kRowWarps)
 };
 
+// Per-row state every warp keeps for the rows lane, lane + 32 (kRowWarps of them): the
+// reference max of the item so far.
+template <class C>
+struct Track {
+    float m[C::kRowWarps];
+};
+
+// a[i] for a register array of one or two values, without dynamic indexing
+template <int K>
+__device__ __forceinline__ float pick(const float (&a)[K], int i) {
+    if constexpr (K == 1) return a[0];
+    else return i ? a[1] : a[0];
+}
+
 // The item's q rows, landed in stage s as kN rows x 9 chunks: dims [0, 64 kQtChunks) go
-// to TMEM (lane r = row r, bf16 pairs), the rest to their tiles in shared memory (a byte
-// copy: both sides are 1 KB aligned, so the 128-byte swizzle carries over).
-template <int kN>
-__device__ __forceinline__ void move_q(const Smem<kN>& sh, const RowCtx& c, uint32_t s) {
-    using C = Cfg<kN>;
+// to TMEM, every lane l holding query row l % (32 kRowWarps) (bf16 pairs), and the rest to
+// shared memory as 128 A rows of the same replication (a byte copy of 128-byte rows:
+// both sides are 1 KB aligned and row l keeps its row % 8, so the swizzle carries over).
+template <class C>
+__device__ __forceinline__ void move_q(const Smem<C>& sh, const RowCtx<C>& c, uint32_t s) {
+    constexpr int kN = C::kN;
     const uint32_t st = sh.stage(s);
-    if (c.warp * 32 < kN) {
+    const int src_row = c.row;                     // < 32 kRowWarps; >= kN reads padding
 #pragma unroll 1
-        for (int ch = 0; ch < C::kQtChunks; ++ch) {
-            uint32_t v[32];
-            const uint32_t rowa = st + ch * C::kTileBytes + (uint32_t)c.tid * 128;
+    for (int ch = 0; ch < C::kQtChunks; ++ch) {
+        uint32_t v[32];
+        const uint32_t rowa = st + ch * C::kTileBytes + (uint32_t)src_row * 128;
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-                const uint4 x = ptx::ld_shared_v4(rowa + (((uint32_t)jj ^ (uint32_t)(c.tid & 7)) * 16));
-                v[4 * jj] = x.x; v[4 * jj + 1] = x.y; v[4 * jj + 2] = x.z; v[4 * jj + 3] = x.w;
-            }
-            ptx::tmem_st32(c.tmem + c.lane_base + C::kColQ + 32 * ch, v);
+        for (int jj = 0; jj < 8; ++jj) {
+            const uint4 x = ptx::ld_shared_v4(rowa + (((uint32_t)jj ^ (uint32_t)(src_row & 7)) * 16));
+            v[4 * jj] = x.x; v[4 * jj + 1] = x.y; v[4 * jj + 2] = x.z; v[4 * jj + 3] = x.w;
         }
-        ptx::tmem_wait_st();
+        ptx::tmem_st32(c.tmem + c.lane_base + C::kColQ + 32 * ch, v);
     }
+    ptx::tmem_wait_st();
     if constexpr (C::kQsChunks > 0) {
-        constexpr uint32_t bytes = C::kQsChunks * C::kTileBytes;
-        const uint32_t src = st + C::kQtChunks * C::kTileBytes;
-        const uint32_t dst = sh.base_u32 + C::kOffQs;
-#pragma unroll 4
-        for (uint32_t o = (uint32_t)c.tid * 16; o < bytes; o += kRowThreads * 16)
-            { const uint4 x = ptx::ld_shared_v4(src + o); ptx::st_shared_v4(dst + o, x.x, x.y, x.z, x.w); }
+        // A row a = tid (all 128 rows), source row a % (32 kRowWarps)
+        const int a = c.tid;
+        const int r = a % (32 * C::kRowWarps);
+#pragma unroll 1
+        for (int ch = 0; ch < C::kQsChunks; ++ch) {
+            const uint32_t src = st + (C::kQtChunks + ch) * C::kTileBytes + (uint32_t)r * 128;
+            const uint32_t dst = sh.base_u32 + C::kOffQs + ch * (C::kARows * 128) + (uint32_t)a * 128;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const uint4 x = ptx::ld_shared_v4(src + u * 16);
+                ptx::st_shared_v4(dst + u * 16, x.x, x.y, x.z, x.w);
+            }
+        }
     }
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before();
 }
 
-// One page step S (the item's j-th page) for this thread.
-template <int kN>
-__device__ __forceinline__ bool row_step(const DecodeParams& p, const Smem<kN>& sh, const RowCtx& c,
-                                         const Item& it, int n_vis, uint32_t j, uint32_t S,
-                                         uint32_t s, float& m_ref, float& l_sum, float& l_rnd) {
-    using C = Cfg<kN>;
-    const uint32_t sb = S & 1u, par = S & 1u;
-    if (!warp_wait_bar(sh, sh.bar(kBarQkDone + sb), (S >> 1) & 1u, 0x51u)) return false;
-    ptx::tc_fence_after();
-    const int page = it.k_lo + (int)j;
-    float x[64];
-    float fac = 1.f;
-    bool need = false;
-    if (c.row_warp) {
-        uint32_t sv[64];
-        ptx::tmem_ld64(c.tmem + c.lane_base + C::kColS + 64 * sb, sv);
-        const int lim = n_vis - page * kBlock;                  // valid tokens [0, lim)
-        const float base = m_ref == -INFINITY ? 0.f : m_ref;
-        const float L2 = p.scale_log2;
-        if (__all_sync(0xffffffffu, lim >= 64)) {
+// FP8 cache: widens a page from staging buffer fidx % 2 into the stage of ring slot g, as
+// the 9-tile swizzled bf16 layout QK and PV read (the rope tile arrives by TMA). Thread t
+// takes token t / 2, dims [256 (t % 2), +256): the scales of its two 128-dim groups, and
+// 256 codes, each read back as the format defines it: E4M3 -> f16 (exact), times the
+// scale in fp32, rounded to bf16 (both nearest-even). Rows past the sequence end are
+// written as zeros (their codes may be anything, NaN included).
+template <class C>
+__device__ __forceinline__ bool dequant(const Smem<C>& sh, const RowCtx<C>& c, const Item& it,
+                                        int page, uint32_t g, uint32_t fidx) {
+    const uint32_t f = fidx % C::kF8Stages, s = g % C::kStages;
+    if (!warp_wait_bar(sh, sh.bar(kBarF8Full + f), (fidx / C::kF8Stages) & 1u, 0x58u)) return false;
+    if (g >= (uint32_t)C::kStages &&
+        !warp_wait_bar(sh, sh.bar(kBarFree + s), ((g / C::kStages) - 1u) & 1u, 0x59u))
+        return false;
+    const int row = c.tid >> 1, half = c.tid & 1;
+    const bool live = page * kBlock + row < it.L;
+    const uint32_t src = sh.f8buf(f) + (uint32_t)row * C::kF8RowBytes;
+    const uint32_t dst = sh.stage(s) + (uint32_t)row * 128;
+    const uint4 scv = ptx::ld_shared_v4(src + 512);            // the row's four group scales
+    const float sc0 = __uint_as_float(half ? scv.z : scv.x);
+    const float sc1 = __uint_as_float(half ? scv.w : scv.y);
 #pragma unroll
-            for (int q = 0; q < 64; ++q) x[q] = fmaf(f32(sv[q]), L2, -base);
-        } else {
+    for (int cc = 0; cc < 4; ++cc) {                           // tile 4 half + cc: 64 dims
+        const float sc = cc < 2 ? sc0 : sc1;
+        const uint32_t tile = dst + (uint32_t)(4 * half + cc) * kBoxBytes;
 #pragma unroll
-            for (int q = 0; q < 64; ++q) x[q] = q < lim ? fmaf(f32(sv[q]), L2, -base) : -INFINITY;
+        for (int h = 0; h < 4; ++h) {                          // 16 codes -> units 2h, 2h+1
+            const uint4 w = ptx::ld_shared_v4(src + (uint32_t)(half * 256 + cc * 64 + h * 16));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            uint32_t o[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t lo = ptx::e4m3x2_to_f16x2((uint16_t)(ws[k] & 0xffffu));
+                const uint32_t hi = ptx::e4m3x2_to_f16x2((uint16_t)(ws[k] >> 16));
+                const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+                const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+                const __nv_bfloat162 r0 = __floats2bfloat162_rn(__fmul_rn(a.x, sc), __fmul_rn(a.y, sc));
+                const __nv_bfloat162 r1 = __floats2bfloat162_rn(__fmul_rn(b.x, sc), __fmul_rn(b.y, sc));
+                o[2 * k] = live ? *reinterpret_cast<const uint32_t*>(&r0) : 0u;
+                o[2 * k + 1] = live ? *reinterpret_cast<const uint32_t*>(&r1) : 0u;
+            }
+            const uint32_t sw = (uint32_t)(row & 7);
+            ptx::st_shared_v4(tile + (((uint32_t)(2 * h) ^ sw) * 16), o[0], o[1], o[2], o[3]);
+            ptx::st_shared_v4(tile + (((uint32_t)(2 * h + 1) ^ sw) * 16), o[4], o[5], o[6], o[7]);
         }
-        float m8[8];
-#pragma unroll
-        for (int a = 0; a < 8; ++a)
-            m8[a] = fmaxf(fmaxf(fmaxf(x[a], x[a + 8]), fmaxf(x[a + 16], x[a + 24])),
-                          fmaxf(fmaxf(x[a + 32], x[a + 40]), fmaxf(x[a + 48], x[a + 56])));
-        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        const float mx_abs = mx + base;
-        const bool raise = m_ref == -INFINITY ? mx_abs > -INFINITY : mx_abs > m_ref + kRescaleLog2;
-        const float m_new = raise ? mx_abs : m_ref;
-        if (m_new != base && m_new != -INFINITY) {
-            const float d = m_new - base;
-#pragma unroll
-            for (int q = 0; q < 64; ++q) x[q] -= d;
-        }
-        need = raise && m_ref != -INFINITY;        // O^T holds earlier pages at m_ref
-        if (need) {
-            fac = ptx::ex2_ftz(m_ref - m_new);
-            l_sum *= fac;
-            l_rnd *= fac;
-        }
-        m_ref = m_new;
-        if (c.tid < 64) sh.facs(par)[c.tid] = fac;
-        if (need) *sh.resc_tag(par) = (int)(S + 1);
     }
+    ptx::fence_proxy_async_smem();           // the widened tiles visible to the MMA
+    warp_arrive(sh.bar(kBarDqFull + s));
+    warp_arrive(sh.bar(kBarF8Free + f));
+    return true;
+}
+
+// One page step S (the item's j-th page) for this thread.
+template <class C>
+__device__ __forceinline__ bool row_step(const DecodeParams& p, const Smem<C>& sh, const RowCtx<C>& c,
+                                         const Item& it, int n_vis, uint32_t j, uint32_t S,
+                                         uint32_t s, Track<C>& tr, float& l_sum, float& l_rnd) {
+    constexpr int kN = C::kN;
+    constexpr int kTok = C::kTok;
+    const uint32_t sb = S % C::kSBufs, par = S & 1u;
+    const uint32_t qpar = C::kSBufs == 2 ? (S >> 1) & 1u : S & 1u;
+    if (!warp_wait_bar(sh, sh.bar(kBarQkDone + sb), qpar, 0x51u)) return false;
+    ptx::tc_fence_after();
+    uint32_t sv[kTok];
+    tmem_ld_cols<kTok>(c.tmem + c.lane_base + C::kColS + 64 * sb + c.copy * kTok, sv);
+    if constexpr (C::kSBufs == 1) {
+        ptx::tc_fence_before();                    // S read out before QK of S+1 rewrites it
+        warp_arrive(sh.bar(kBarSFree));
+    }
+    const int page = it.k_lo + (int)j;
+    const int lim = n_vis - page * kBlock - c.copy * kTok;    // valid tokens of the slice [0, lim)
+    const float m_own = pick(tr.m, c.own);
+    const float base = m_own == -INFINITY ? 0.f : m_own;
+    const float L2 = p.scale_log2;
+    float x[kTok];
+    if (__all_sync(0xffffffffu, lim >= kTok)) {
+#pragma unroll
+        for (int q = 0; q < kTok; ++q) x[q] = fmaf(f32(sv[q]), L2, -base);
+    } else {
+#pragma unroll
+        for (int q = 0; q < kTok; ++q) x[q] = q < lim ? fmaf(f32(sv[q]), L2, -base) : -INFINITY;
+    }
+    float mx = x[0];
+#pragma unroll
+    for (int q = 1; q < kTok; ++q) mx = fmaxf(mx, x[q]);
+    sh.pmax(par, c.copy)[c.row] = mx + base;
     warp_arrive(sh.bar(kBarDecide));
     if (!warp_wait_bar(sh, sh.bar(kBarDecide), par, 0x52u)) return false;
-    const bool resc = *sh.resc_tag(par) == (int)(S + 1);
-    if (resc || S > 0) {
+    // every tracked row's page max, reference update and O^T factor (identical in every
+    // warp: the same maxima and the same history)
+    float fac[C::kRowWarps];
+    bool any = false;
+#pragma unroll
+    for (int k = 0; k < C::kRowWarps; ++k) {
+        const int r = c.lane + 32 * k;
+        float pm = -INFINITY;
+#pragma unroll
+        for (int cp = 0; cp < C::kCopies; ++cp)
+            pm = fmaxf(pm, *reinterpret_cast<volatile float*>(&sh.pmax(par, cp)[r]));
+        const float mo = tr.m[k];
+        const bool raise = mo == -INFINITY ? pm > -INFINITY : pm > mo + kRescaleLog2;
+        const float mn = raise ? pm : mo;
+        const bool need = raise && mo != -INFINITY;           // O^T holds pages at mo
+        fac[k] = need ? ptx::ex2_ftz(mo - mn) : 1.f;
+        any |= need;
+        tr.m[k] = mn;
+    }
+    const float m_new = pick(tr.m, c.own);
+    if (m_new != base && m_new != -INFINITY) {
+        const float d = m_new - base;
+#pragma unroll
+        for (int q = 0; q < kTok; ++q) x[q] -= d;
+    }
+    l_sum *= pick(fac, c.own);
+    l_rnd *= pick(fac, c.own);
+    any = __any_sync(0xffffffffu, any);
+    if (any || S > 0) {
         // PV of step S-1 must be done: before O^T is rescaled, and before P is rewritten
         if (!warp_wait_bar(sh, sh.bar(kBarPvDone), (S - 1) & 1u, 0x53u)) return false;
         ptx::tc_fence_after();
     }
-    if (resc) {
-        // scale the O^T columns of rows that raised their reference (factor 1 elsewhere)
-        const float* f = sh.facs(par);
+    if (any) {
+        // scale O^T column r (query row r) by its row's factor; the factor of row r is
+        // held by lane r % 32 (tracked index r / 32)
 #pragma unroll 1
-        for (int i = 0; i < 4; ++i) {
+        for (int cc = 0; cc < kN; cc += 16) {
+            float f[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int r = cc + e;
+                f[e] = __shfl_sync(0xffffffffu, pick(fac, r >> 5), r & 31);
+            }
 #pragma unroll 1
-            for (int cc = 0; cc < kN; cc += 16) {
+            for (int i = 0; i < 4; ++i) {
                 uint32_t v[16];
                 const uint32_t a = c.tmem + c.lane_base + C::kColO + kN * i + cc;
                 ptx::tmem_ld16(a, v);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(f32(v[e]) * f[cc + e]);
+                for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(f32(v[e]) * f[e]);
                 ptx::tmem_st16(a, v);
             }
         }
         ptx::tmem_wait_st();
     }
-    if (c.row_warp) {
-        uint32_t pk[32];
+    {
+        uint32_t pk[kTok / 2];
         float rs0 = 0.f, rs1 = 0.f, rr0 = 0.f, rr1 = 0.f;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < kTok / 2; ++q) {
             const float p0 = ptx::ex2_ftz(x[2 * q]);
             const float p1 = ptx::ex2_ftz(x[2 * q + 1]);
             rs0 += p0;
@@ -461,19 +682,22 @@ __device__ __forceinline__ bool row_step(const DecodeParams& p, const Smem<kN>& 
         }
         l_sum += rs0 + rs1;
         l_rnd += rr0 + rr1;
-        if (c.tid < kN) {
-            // row of P: 64 tokens = 8 chunks of 16 B, K-major, 128-byte swizzle
-            const uint32_t prow = sh.base_u32 + C::kOffP + (uint32_t)c.tid * 128;
+        if (c.row < kN) {
+            // this slice of the row of P: tokens [copy kTok, +kTok) = 16-byte units
+            // [copy kTok / 8, +kTok / 8) of the 128-byte row, K-major, 128-byte swizzle
+            const uint32_t prow = sh.base_u32 + C::kOffP + (uint32_t)c.row * 128;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-                ptx::st_shared_v4(prow + (((uint32_t)cc ^ (uint32_t)(c.tid & 7)) * 16), pk[4 * cc],
-                                  pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+            for (int u = 0; u < kTok / 8; ++u) {
+                const uint32_t unit = (uint32_t)(c.copy * (kTok / 8) + u);
+                ptx::st_shared_v4(prow + ((unit ^ (uint32_t)(c.row & 7)) * 16), pk[4 * u],
+                                  pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            }
         }
     }
     // V rows past the sequence end (they may hold stale or NaN data, and P = 0 would not
     // cancel NaN): zero them in the stage. QK of this step, their only other reader, is done.
     const int tail = it.L - page * kBlock;
-    if (tail < kBlock) {
+    if (!C::kF8 && tail < kBlock) {
         const uint32_t st = sh.stage(s);
         const int units = (kBlock - tail) * 64;                 // 8 chunks x 8 x 16 B per row
         for (int q = c.tid; q < units; q += kRowThreads) {
@@ -487,32 +711,43 @@ __device__ __forceinline__ bool row_step(const DecodeParams& p, const Smem<kN>& 
     return true;
 }
 
-// Epilogue of an item: the row threads post 1/l and write the lse; then every thread (TMEM
-// lane = latent dim) writes its dim of each real row, normalised, as bf16 `out`, fp32
-// `out_f32` or the fp32 split partial.
-template <int kN>
-__device__ __forceinline__ bool epilogue(const DecodeParams& p, const Smem<kN>& sh, const RowCtx& c,
-                                         const Item& it, float m_ref, float l_sum, float l_rnd,
+// Epilogue of an item: the partial row sums of the token slices meet in shared memory;
+// the threads of copy 0 post 1/l and write the lse; then every thread (TMEM lane = latent
+// dim) writes its dim of each real row, normalised, as bf16 `out`, fp32 `out_f32` or the
+// fp32 split partial.
+template <class C>
+__device__ __forceinline__ bool epilogue(const DecodeParams& p, const Smem<C>& sh, const RowCtx<C>& c,
+                                         const Item& it, float m_row, float l_sum, float l_rnd,
                                          uint32_t last_step, uint32_t epi_index) {
-    using C = Cfg<kN>;
+    constexpr int kN = C::kN;
     const bool final_out = it.n_chunks == 1;
     const bool have_ws = it.part < p.max_chunks;
-    if (c.row_warp && c.tid < 64) {
-        const bool empty = !(l_sum > 0.f);
-        sh.inv_l()[c.tid] = empty ? 0.f : 1.f / l_rnd;
-        if (c.tid < p.rows) {
-            const float lse2 = empty ? -INFINITY : m_ref + __log2f(l_sum);
+    sh.psum(0, c.copy)[c.row] = l_sum;
+    sh.psum(1, c.copy)[c.row] = l_rnd;
+    warp_arrive(sh.bar(kBarEpi));
+    if (!warp_wait_bar(sh, sh.bar(kBarEpi), (2 * epi_index) & 1u, 0x54u)) return false;
+    if (c.copy == 0) {
+        float lt = 0.f, lr = 0.f;
+#pragma unroll
+        for (int cp = 0; cp < C::kCopies; ++cp) {
+            lt += *reinterpret_cast<volatile float*>(&sh.psum(0, cp)[c.row]);
+            lr += *reinterpret_cast<volatile float*>(&sh.psum(1, cp)[c.row]);
+        }
+        const bool empty = !(lt > 0.f);
+        sh.inv_l()[c.row] = empty ? 0.f : 1.f / lr;
+        if (c.row < p.rows) {
+            const float lse2 = empty ? -INFINITY : m_row + __log2f(lt);
             if (final_out) {
-                const int qi = c.tid / p.h_q, h = c.tid % p.h_q;
+                const int qi = c.row / p.h_q, h = c.row % p.h_q;
                 p.lse[((size_t)it.b * p.h_q + h) * p.s_q + qi] = empty ? -INFINITY : lse2 * kLn2;
             } else if (have_ws) {
-                p.ws_lse[(size_t)it.part * kTileRows + c.tid] = lse2;
+                p.ws_lse[(size_t)it.part * kTileRows + c.row] = lse2;
             }
         }
     }
     if (!final_out && !have_ws && c.tid == 0) record_error(kErrWorkspace, (uint32_t)it.v & 0xffffffu);
     warp_arrive(sh.bar(kBarEpi));
-    if (!warp_wait_bar(sh, sh.bar(kBarEpi), epi_index & 1u, 0x54u)) return false;
+    if (!warp_wait_bar(sh, sh.bar(kBarEpi), (2 * epi_index + 1) & 1u, 0x56u)) return false;
     if (!warp_wait_bar(sh, sh.bar(kBarPvDone), last_step & 1u, 0x55u)) return false;
     ptx::tc_fence_after();
     const float* inv_l = sh.inv_l();
@@ -545,20 +780,23 @@ __device__ __forceinline__ bool epilogue(const DecodeParams& p, const Smem<kN>& 
     return true;
 }
 
-template <int kN>
-__device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<kN>& sh, uint32_t tmem) {
-    using C = Cfg<kN>;
-    RowCtx c;
+template <class C>
+__device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<C>& sh, uint32_t tmem) {
+    constexpr int kN = C::kN;
+    RowCtx<C> c;
     c.tmem = tmem;
     c.tid = (int)threadIdx.x;
     c.warp = c.tid >> 5;
     c.lane = c.tid & 31;
     c.lane_base = (uint32_t)(c.warp * 32) << 16;
-    c.row_warp = c.warp * 32 < p.rows;
+    c.copy = c.warp / C::kRowWarps;
+    c.own = c.warp % C::kRowWarps;
+    c.row = c.own * 32 + c.lane;
     ItemIter iter(p, (int)blockIdx.x, (int)gridDim.x);
     Item it, prev;
     uint32_t g = 0, gs = 0, items = 0;
-    float m_ref = -INFINITY, l_sum = 0.f, l_rnd = 0.f;
+    Track<C> tr;
+    float l_sum = 0.f, l_rnd = 0.f;
     float prev_m = -INFINITY, prev_l = 0.f, prev_r = 0.f;
     bool have_prev = false;
     while (iter.next(it)) {
@@ -573,21 +811,30 @@ __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<kN>& 
         if (have_prev) {
             if (!epilogue(p, sh, c, prev, prev_m, prev_l, prev_r, gs - 1, items - 1)) return;
         }
-        const bool row_valid = c.tid < p.rows;
-        const int qi = row_valid ? c.tid / p.h_q : 0;
+        const bool row_valid = c.row < p.rows;
+        const int qi = row_valid ? c.row / p.h_q : 0;
         const int n_vis = row_valid ? visible_tokens(it.L, p.s_q, qi, p.causal) : 0;
-        m_ref = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < C::kRowWarps; ++k) tr.m[k] = -INFINITY;
         l_sum = 0.f;
         l_rnd = 0.f;
         const uint32_t n = (uint32_t)it.pages();
+        // FP8 cache: widen the item's first page now and page j + 1 before the softmax of
+        // page j, so QK of the next page finds its operands ready
+        if constexpr (C::kF8) {
+            if (!dequant(sh, c, it, it.k_lo, g, gs)) return;
+        }
         for (uint32_t j = 0; j < n; ++j) {
-            if (!row_step(p, sh, c, it, n_vis, j, gs + j, (g + j) % C::kStages, m_ref, l_sum, l_rnd))
+            if constexpr (C::kF8) {
+                if (j + 1 < n && !dequant(sh, c, it, it.k_lo + (int)j + 1, g + j + 1, gs + j + 1)) return;
+            }
+            if (!row_step(p, sh, c, it, n_vis, j, gs + j, (g + j) % C::kStages, tr, l_sum, l_rnd))
                 return;
         }
         g += n;
         gs += n;
         prev = it;
-        prev_m = m_ref;
+        prev_m = pick(tr.m, c.own);
         prev_l = l_sum;
         prev_r = l_rnd;
         have_prev = true;
@@ -596,13 +843,15 @@ __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<kN>& 
     if (have_prev) epilogue(p, sh, c, prev, prev_m, prev_l, prev_r, gs - 1, items - 1);
 }
 
-template <int kN>
+// tm_page: the bf16 pool's pages, or for an FP8 cache its rows' codes and scales;
+// tm_rope: FP8 cache only, the rope dims of its rows as bf16 (unused otherwise).
+template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
-              const __grid_constant__ CUtensorMap tm_q) {
-    using C = Cfg<kN>;
+              const __grid_constant__ CUtensorMap tm_rope, const __grid_constant__ CUtensorMap tm_q) {
+    constexpr int kN = C::kN;
     extern __shared__ uint8_t smem_raw[];
-    Smem<kN> sh;
+    Smem<C> sh;
     {
         const uint32_t raw = ptx::smem_u32(smem_raw);
         const uint32_t aligned = (raw + 1023u) & ~1023u;
@@ -620,18 +869,23 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
         ptx::mbar_init(sh.bar(kBarQkDone + 1), 1);
         ptx::mbar_init(sh.bar(kBarPvDone), 1);
         ptx::mbar_init(sh.bar(kBarPReady), 4);
+        ptx::mbar_init(sh.bar(kBarSFree), 4);
         ptx::mbar_init(sh.bar(kBarQReady), 4);
         ptx::mbar_init(sh.bar(kBarOFree), 4);
         ptx::mbar_init(sh.bar(kBarDecide), 4);
         ptx::mbar_init(sh.bar(kBarEpi), 4);
         ptx::mbar_init(sh.bar(kBarDrain), 1);
         ptx::mbar_init(sh.bar(kBarStall), 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(sh.bar(kBarF8Full + i), 1);
+            ptx::mbar_init(sh.bar(kBarF8Free + i), 4);
+        }
+        for (int i = 0; i < kMaxStages; ++i) ptx::mbar_init(sh.bar(kBarDqFull + i), 4);
         *sh.abort_flag() = 0;
-        *sh.resc_tag(0) = 0;
-        *sh.resc_tag(1) = 0;
         ptx::fence_mbarrier_init_cluster();
         ptx::prefetch_tensormap(&tm_page);
         ptx::prefetch_tensormap(&tm_q);
+        if (C::kF8) ptx::prefetch_tensormap(&tm_rope);
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc(ptx::smem_u32(sh.tmem_slot()), kTmemCols);
@@ -643,11 +897,14 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
     const uint32_t tmem = *sh.tmem_slot();
 
     if (warp < 4) {
-        run_rows<kN>(p, sh, tmem);
+        run_rows<C>(p, sh, tmem);
     } else if (warp == kWarpProducer) {
-        if (lane == 0) run_producer<kN>(p, sh, &tm_page, &tm_q);
+        if (lane == 0) {
+            if constexpr (C::kF8) run_producer_f8<C>(p, sh, &tm_page, &tm_rope, &tm_q);
+            else run_producer<C>(p, sh, &tm_page, &tm_q);
+        }
     } else if (warp == kWarpMma) {
-        if (lane == 0) run_mma<kN>(p, sh, tmem);
+        if (lane == 0) run_mma<C>(p, sh, tmem);
     }
     ptx::tc_fence_before();
     __syncthreads();

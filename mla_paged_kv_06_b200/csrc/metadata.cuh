@@ -41,7 +41,7 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* smem
     return total;
 }
 
-// metadata: header {num_units, tiles, batch, h_q, s_q, unit_cost, 0, 0} then one
+// metadata: header {num_units, tiles, batch, h_q, s_q, unit_cost, overhead, 0} then one
 // {v_begin, page_begin, v_end, page_end, chunk_begin, 0, 0, 0} per unit.
 // num_splits holds the cumulative costs C[v] while the units are located, then is
 // overwritten with the chunk prefix.
@@ -56,6 +56,7 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
     __shared__ int64_t s_total;
     extern __shared__ int32_t dyn[];
     const int V = batch * tiles;
+    const int overhead = overhead_pages(h_q, s_q);
     int32_t* Cs = in_smem ? dyn : num_splits;               // cumulative costs C[0..V]
     int32_t* Ps = in_smem ? dyn + V + 1 : nullptr;          // pages per sequence
     if (in_smem) {
@@ -75,7 +76,7 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
     int64_t carry = 0;
     for (int base = 0; base < V; base += blockDim.x) {
         int v = base + threadIdx.x;
-        int64_t cost = v < V ? (int64_t)kOverheadPages + pages(v) : 0;
+        int64_t cost = v < V ? (int64_t)overhead + pages(v) : 0;
         int64_t pre;
         int64_t tot = block_exclusive_scan(cost, warp_sums, &pre);
         int64_t c = carry + pre;
@@ -98,11 +99,11 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
     // Phase 2: one thread per unit locates its first and one-past-last page.
     for (int u = threadIdx.x; u < num_units; u += blockDim.x) {
         int vb, kb, ve, ke;
-        locate((int64_t)u * W, C, pages, V, kOverheadPages, &vb, &kb);
-        locate((int64_t)(u + 1) * W, C, pages, V, kOverheadPages, &ve, &ke);
+        locate((int64_t)u * W, C, pages, V, overhead, &vb, &kb);
+        locate((int64_t)(u + 1) * W, C, pages, V, overhead, &ve, &ke);
         int chunk = 0;
         if (vb < V && (vb != ve || kb != ke))
-            chunk = u - unit_of(C(vb) + kOverheadPages, W);
+            chunk = u - unit_of(C(vb) + overhead, W);
         int32_t* m = metadata + kMetaInts * (u + 1);
         m[0] = vb; m[1] = kb; m[2] = ve; m[3] = ke; m[4] = chunk;
         m[5] = 0; m[6] = 0; m[7] = 0;
@@ -111,7 +112,7 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
         metadata[0] = num_units; metadata[1] = tiles; metadata[2] = batch;
         metadata[3] = h_q; metadata[4] = s_q;
         metadata[5] = (int32_t)(W > 0x7fffffffLL ? 0x7fffffff : W);
-        metadata[6] = 0; metadata[7] = 0;
+        metadata[6] = overhead; metadata[7] = 0;
     }
     __syncthreads();
 
@@ -120,7 +121,7 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
     carry = 0;
     for (int base = 0; base < V; base += blockDim.x) {
         int v = base + threadIdx.x;
-        int n = v < V ? chunks_of(C(v), pages(v), W, kOverheadPages) : 0;
+        int n = v < V ? chunks_of(C(v), pages(v), W, overhead) : 0;
         int64_t pre;
         int64_t tot = block_exclusive_scan(n, warp_sums, &pre);   // also a barrier
         if (v < V) num_splits[v] = (int32_t)(carry + pre);

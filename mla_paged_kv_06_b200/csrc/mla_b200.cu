@@ -41,11 +41,13 @@ bool shape_ok(int batch, int h_q, int s_q) {
            s_q >= 1 && s_q <= MLA_MAX_S_Q && h_q * s_q <= MLA_MAX_ROWS;
 }
 
-// Query rows per sequence up to which the 1-CTA kernel (decode_solo.cuh) runs; above it
-// the 2-CTA kernel (decode_pair.cuh) splits 128-row tiles over two SMs.
-constexpr int kSoloMaxRows = 64;
-
+// Up to kSoloMaxRows query rows per sequence the 1-CTA kernel (decode_solo.cuh) runs;
+// above it the 2-CTA kernel (decode_pair.cuh) splits 128-row tiles over two SMs.
 bool use_solo(int h_q, int s_q) { return h_q * s_q <= kSoloMaxRows; }
+
+// Query rows per sequence the FP8-cache decode takes: its two 33 KB staging buffers fit
+// beside two bf16 stages only for the 1-CTA kernel's 16- and 32-row layouts.
+constexpr int kFp8MaxRows = 32;
 
 // Work units a schedule for num_sms SMs may use, before the device cap: one per SM for
 // the 1-CTA kernel, one per SM pair for the 2-CTA kernel.
@@ -144,15 +146,15 @@ int device_pairs(int dev) {
     return pairs;
 }
 
-template <int kN>
+template <class C>
 bool prepare_solo_kernel(int dev) {
     static std::mutex mu;
     static std::vector<char> done;
     std::lock_guard<std::mutex> lock(mu);
     if ((int)done.size() <= dev) done.resize(dev + 1, 0);
     if (done[dev]) return true;
-    if (cudaFuncSetAttribute(solo::decode_kernel<kN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)solo::Cfg<kN>::kSmemAlloc) != cudaSuccess)
+    if (cudaFuncSetAttribute(solo::decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C::kSmemAlloc) != cudaSuccess)
         return false;
     done[dev] = 1;
     return true;
@@ -172,9 +174,9 @@ int device_solo_ctas(int dev) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return -1;
     int ctas = sms < 1 ? 1 : sms;
-    if (prepare_solo_kernel<64>(dev)) {
+    if (prepare_solo_kernel<solo::Cfg<64>>(dev)) {
         int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, solo::decode_kernel<64>,
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, solo::decode_kernel<solo::Cfg<64>>,
                                                           solo::kThreads,
                                                           solo::Cfg<64>::kSmemAlloc) == cudaSuccess &&
             per_sm >= 1 && per_sm * sms < ctas)
@@ -323,12 +325,59 @@ mla_status launch_combine(const DecodeParams& p, cudaStream_t s) {
 template <int kN>
 mla_status launch_solo(const DecodeParams& p, const void* q, const void* kcache, int num_blocks,
                        int ctas, int dev, cudaStream_t s) {
-    if (!prepare_solo_kernel<kN>(dev)) return MLA_ERR_CUDA;
+    using C = solo::Cfg<kN>;
+    if (!prepare_solo_kernel<C>(dev)) return MLA_ERR_CUDA;
     CUtensorMap tm_page, tm_q;
     if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
         !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
         return MLA_ERR_CUDA;
-    solo::decode_kernel<kN><<<ctas, solo::kThreads, solo::Cfg<kN>::kSmemAlloc, s>>>(p, tm_page, tm_q);
+    solo::decode_kernel<C><<<ctas, solo::kThreads, C::kSmemAlloc, s>>>(p, tm_page, tm_page, tm_q);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// FP8 cache ([num_blocks][64][656] bytes, rows of MLA_FP8_ROW_BYTES): the rows' codes and
+// scales as a 3-D byte view {16 bytes, 41 units of 16 bytes, rows} with box {16, 33, 64}
+// (a page's 64 rows x 528 bytes, dense), and their rope dims as a 2-D bf16 view {64
+// elements, rows} starting 528 bytes into the pool, row stride 656 bytes, box {64, 64},
+// 128-byte swizzle (one swizzled tile, as the bf16 pool's rope chunk lands).
+bool make_f8_maps(CUtensorMap* codes, CUtensorMap* rope, const void* kc8, int num_blocks) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t rows = (cuuint64_t)num_blocks * kBlock;
+    {
+        const cuuint64_t dims[3] = {16, MLA_FP8_ROW_BYTES / 16, rows};
+        const cuuint64_t strides[2] = {16, MLA_FP8_ROW_BYTES};
+        const cuuint32_t box[3] = {16, 33, (cuuint32_t)kBlock};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (fn(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(kc8), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[2] = {64, rows};
+        const cuuint64_t strides[1] = {MLA_FP8_ROW_BYTES};
+        const cuuint32_t box[2] = {64, (cuuint32_t)kBlock};
+        const cuuint32_t estr[2] = {1, 1};
+        void* base = const_cast<char*>(static_cast<const char*>(kc8)) + 528;
+        if (fn(rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    return true;
+}
+
+template <int kN>
+mla_status launch_solo_f8(const DecodeParams& p, const void* q, const void* kc8, int num_blocks,
+                          int ctas, int dev, cudaStream_t s) {
+    using C = solo::Cfg<kN, true>;
+    if (!prepare_solo_kernel<C>(dev)) return MLA_ERR_CUDA;
+    CUtensorMap tm_codes, tm_rope, tm_q;
+    if (!make_f8_maps(&tm_codes, &tm_rope, kc8, num_blocks) ||
+        !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
+        return MLA_ERR_CUDA;
+    solo::decode_kernel<C><<<ctas, solo::kThreads, C::kSmemAlloc, s>>>(p, tm_codes, tm_rope, tm_q);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -545,6 +594,33 @@ mla_status mla_decode_fwd_noalloc(const uint16_t* q, const uint16_t* kcache, int
     return launch_decode(p, q, kcache, num_blocks, (cudaStream_t)stream);
 }
 
+mla_status mla_decode_fwd_fp8(const uint16_t* q, const uint8_t* kcache_fp8, int num_blocks,
+                              const int32_t* block_table, int max_blocks, const int32_t* seqlens,
+                              int batch, int s_q, int h_q, float scale, int causal,
+                              const int32_t* metadata, const int32_t* num_splits,
+                              void* workspace, size_t workspace_bytes, uint16_t* out, float* lse,
+                              void* stream) {
+    // the validation of mla_decode_fwd (the cache pointer takes the bf16 pool's checks)
+    mla_status st = validate_decode(q, reinterpret_cast<const uint16_t*>(kcache_fp8), num_blocks,
+                                    block_table, max_blocks, seqlens, batch, s_q, h_q, scale,
+                                    causal, metadata, num_splits, workspace, workspace_bytes, out,
+                                    lse);
+    if (st != MLA_OK) return st;
+    if (h_q * s_q > kFp8MaxRows) return MLA_ERR_UNSUPPORTED;
+    DecodeParams p = make_params(q, reinterpret_cast<const uint16_t*>(kcache_fp8), num_blocks,
+                                 block_table, max_blocks, seqlens, batch, s_q, h_q, scale, causal,
+                                 metadata, num_splits, workspace, workspace_bytes, out, lse);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+    const int ctas = device_solo_ctas(dev);
+    if (ctas < 1) return MLA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    st = p.rows <= 16 ? launch_solo_f8<16>(p, q, kcache_fp8, num_blocks, ctas, dev, s)
+                      : launch_solo_f8<32>(p, q, kcache_fp8, num_blocks, ctas, dev, s);
+    if (st != MLA_OK) return st;
+    return launch_combine(p, s);
+}
+
 mla_status mla_kv_append(const uint16_t* kv_new, int s_new, const int32_t* block_table,
                          int max_blocks, const int32_t* seqlens, int batch, uint16_t* kcache,
                          int num_blocks, void* stream) {
@@ -597,12 +673,13 @@ mla_status mla_plan_host(const int32_t* seqlens_host, int batch, int h_q, int s_
     if (!shape_ok(batch, h_q, s_q)) return MLA_ERR_UNSUPPORTED;
     const int tiles = num_tiles(h_q, s_q);
     const int V = batch * tiles;
+    const int overhead = overhead_pages(h_q, s_q);
     std::vector<int> nblk(V);
     std::vector<int64_t> C(V + 1, 0);
     for (int v = 0; v < V; ++v) {
         const int L = seqlens_host[v % batch];
         nblk[v] = pages_of(L < 0 ? 0 : L);
-        C[v + 1] = C[v] + kOverheadPages + nblk[v];
+        C[v + 1] = C[v] + overhead + nblk[v];
     }
     if (C[V] > 0x7fffffffLL) return MLA_ERR_UNSUPPORTED;
     const int64_t W = unit_cost(C[V], num_units);
@@ -610,21 +687,21 @@ mla_status mla_plan_host(const int32_t* seqlens_host, int batch, int h_q, int s_
     auto pages = [&](int v) { return nblk[v]; };
     for (int u = 0; u < num_units; ++u) {
         int vb, kb, ve, ke;
-        locate((int64_t)u * W, cost, pages, V, kOverheadPages, &vb, &kb);
-        locate((int64_t)(u + 1) * W, cost, pages, V, kOverheadPages, &ve, &ke);
+        locate((int64_t)u * W, cost, pages, V, overhead, &vb, &kb);
+        locate((int64_t)(u + 1) * W, cost, pages, V, overhead, &ve, &ke);
         int chunk = 0;
-        if (vb < V && (vb != ve || kb != ke)) chunk = u - unit_of(C[vb] + kOverheadPages, W);
+        if (vb < V && (vb != ve || kb != ke)) chunk = u - unit_of(C[vb] + overhead, W);
         int32_t* m = metadata_host + kMetaInts * (u + 1);
         m[0] = vb; m[1] = kb; m[2] = ve; m[3] = ke; m[4] = chunk;
         m[5] = 0; m[6] = 0; m[7] = 0;
     }
     metadata_host[0] = num_units; metadata_host[1] = tiles; metadata_host[2] = batch;
     metadata_host[3] = h_q; metadata_host[4] = s_q; metadata_host[5] = (int32_t)W;
-    metadata_host[6] = 0; metadata_host[7] = 0;
+    metadata_host[6] = overhead; metadata_host[7] = 0;
     int32_t acc = 0;
     for (int v = 0; v < V; ++v) {
         num_splits_host[v] = acc;
-        acc += chunks_of(C[v], nblk[v], W, kOverheadPages);
+        acc += chunks_of(C[v], nblk[v], W, overhead);
     }
     num_splits_host[V] = acc;
     return MLA_OK;

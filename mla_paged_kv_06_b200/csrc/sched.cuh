@@ -27,9 +27,17 @@ namespace mla {
 constexpr int kBlock = 64;
 constexpr int kTileRows = 128;
 // Fixed cost of one work sequence in page units: loading its query tile, refilling the
-// pipeline and its epilogue. Measured on B200 with the split kernel, an item boundary
-// costs about as much as three and a half pages.
+// pipeline and its epilogue. Measured on B200: an item boundary of the 2-CTA kernel costs
+// about as much as three and a half pages; one of the 1-CTA kernel (sequences of at most
+// kSoloMaxRows query rows), whose q rows ride in a slot of the page ring and whose
+// epilogue overlaps the next item's first QK, about half a page.
 constexpr int kOverheadPages = 3;
+constexpr int kOverheadPagesSolo = 1;
+constexpr int kSoloMaxRows = 64;
+
+MLA_HD int overhead_pages(int h_q, int s_q) {
+    return h_q * s_q <= kSoloMaxRows ? kOverheadPagesSolo : kOverheadPages;
+}
 constexpr int kMetaInts = 8;
 // Smallest per-unit cost: a split costs a partial tile write and a combine read, so
 // cutting work finer than a few pages loses more than it balances.

@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
                                          vp, vp, vp, vp, vp]),
         "mla_decode_fwd_partial": (i32, [vp, vp, i32, vp, i32, vp, i32, i32, i32, f32, i32,
                                          vp, vp, vp, sz, vp, vp, vp]),
+        "mla_decode_fwd_fp8": (i32, [vp, vp, i32, vp, i32, vp, i32, i32, i32, f32, i32,
+                                     vp, vp, vp, sz, vp, vp, vp]),
         "mla_combine_partials": (i32, [vp, vp, i32, i32, i32, i32, vp, vp, vp]),
         "mla_kv_append": (i32, [vp, i32, vp, i32, vp, i32, vp, i32, vp]),
         "mla_kv_append_fp8": (i32, [vp, i32, vp, i32, vp, i32, vp, i32, vp]),
@@ -158,7 +160,11 @@ def _decode(fn_name, q, kcache, block_table, seqlens, scale, causal, metadata, n
             workspace=None, out=None, lse=None, stream=None, num_sms=None,
             out_dtype=torch.bfloat16):
     assert q.is_cuda and q.dtype == torch.bfloat16 and q.dim() == 4 and q.is_contiguous()
-    assert kcache.dtype == torch.bfloat16 and kcache.is_contiguous()
+    if fn_name == "mla_decode_fwd_fp8":
+        assert kcache.dtype == torch.uint8 and kcache.dim() == 3 and kcache.shape[2] == MLA_FP8_ROW_BYTES
+    else:
+        assert kcache.dtype == torch.bfloat16
+    assert kcache.is_contiguous()
     assert block_table.dtype == torch.int32 and block_table.is_contiguous()
     batch, s_q, h_q, _ = q.shape
     num_blocks = kcache.shape[0]
@@ -186,6 +192,15 @@ def mla_decode_fwd(q, kcache, block_table, seqlens, scale, causal, metadata, num
     lse fp32 [b,h_q,s_q])."""
     return _decode("mla_decode_fwd", q, kcache, block_table, seqlens, scale, causal, metadata,
                    num_splits, workspace, out, lse, stream, num_sms)
+
+
+def mla_decode_fwd_fp8(q, kcache_fp8, block_table, seqlens, scale, causal, metadata,
+                       num_splits, workspace=None, out=None, lse=None, stream=None,
+                       num_sms=None):
+    """Paged MLA decode over an FP8 latent cache (uint8 [num_blocks, 64, 656], the row
+    format of mla_kv_append_fp8). Returns (out bf16 [b,s_q,h_q,512], lse fp32 [b,h_q,s_q])."""
+    return _decode("mla_decode_fwd_fp8", q, kcache_fp8, block_table, seqlens, scale, causal,
+                   metadata, num_splits, workspace, out, lse, stream, num_sms)
 
 
 def mla_decode_fwd_partial(q, kcache, block_table, seqlens, scale, causal, metadata,

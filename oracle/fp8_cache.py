@@ -166,7 +166,20 @@ def dequantize_cache(fp8_cache) -> np.ndarray:
     return dequantize_rows(q.reshape(-1, ROW_BYTES)).reshape(nb, 64, 1, LATENT + ROPE)
 
 
-def decode_fp8(q, fp8_cache, block_table, seqlens, scale: float, causal: bool):
-    """Exact decode attention over the dequantized FP8 cache (fp64)."""
+def decode_fp8(q, fp8_cache, block_table, seqlens, scale: float, causal: bool,
+               batch_indices=None):
+    """Exact decode attention over the read-back FP8 cache (fp64), for all sequences or
+    those in `batch_indices`. Only the pages those sequences own are read back (the
+    others are left NaN, and the bf16 oracle never reads a page a sequence does not own)."""
     from .mla_decode import decode
-    return decode(q, dequantize_cache(fp8_cache), block_table, seqlens, scale, causal)
+    q8 = np.asarray(fp8_cache, dtype=np.uint8)
+    nb = q8.shape[0]
+    idx = range(len(seqlens)) if batch_indices is None else list(batch_indices)
+    lens = np.asarray(seqlens, dtype=np.int64)
+    bt = np.asarray(block_table, dtype=np.int64)
+    used = sorted({int(bt[b][j]) for b in idx for j in range((int(lens[b]) + 63) // 64)})
+    deq = np.full((nb, 64, 1, LATENT + ROPE), np.nan)
+    if used:
+        deq[used] = dequantize_rows(q8[used].reshape(-1, ROW_BYTES)).reshape(len(used), 64, 1,
+                                                                             LATENT + ROPE)
+    return decode(q, deq, block_table, seqlens, scale, causal, batch_indices=batch_indices)

@@ -152,7 +152,11 @@ def test_schedule_random_and_balanced():
         meta, ns = mla.mla_plan_host(lens, h_q, s_q, U)
         seen, nblk = _walk(meta, ns, lens, h_q, s_q)
         W = int(meta[5])
-        total = sum(3 + n for n in nblk)          # 3 pages of fixed cost per work sequence
+        # fixed cost per work sequence, in pages: 1 for the 1-CTA kernel (at most 64 query
+        # rows per sequence), 3 for the 2-CTA kernel; the header records it
+        overhead = 1 if h_q * s_q <= 64 else 3
+        assert int(meta[6]) == overhead
+        total = sum(overhead + n for n in nblk)
         assert W == max(-(-total // U), 4)
         # no unit owns more than W pages: the largest unit is within one overhead of ideal
         per_unit = [0] * U
