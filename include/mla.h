@@ -301,10 +301,11 @@ mla_status mla_kv_append_fp8(const uint16_t* kv_new, int s_new, const int32_t* b
  *               16-byte aligned (read)
  *   every other argument as for mla_decode_fwd, with metadata, num_splits and the
  *   workspace size from the same calls for the same shapes.
- * Supported: s_q * h_q <= 32 (the kernel's two 33 KB staging buffers fit beside its
- * bf16 stages only for up to 32 query rows); larger row counts return
- * MLA_ERR_UNSUPPORTED before any launch. The 1-CTA kernel widens each page into bf16 in
- * shared memory before its QK; codes of rows past a sequence's end are never read.
+ * Supported: s_q * h_q <= 64, the row counts of the 1-CTA kernel that runs it; larger
+ * row counts return MLA_ERR_UNSUPPORTED before any launch. The kernel lands each page's
+ * codes, scales and rope dims in one shared-memory stage and widens the codes to bf16 in
+ * place before the page's QK; rows past a sequence's end widen to zeros whatever their
+ * bytes hold (NaN codes or scales included).
  */
 mla_status mla_decode_fwd_fp8(const uint16_t* q, const uint8_t* kcache_fp8, int num_blocks,
                               const int32_t* block_table, int max_blocks,

@@ -57,6 +57,13 @@ constexpr uint32_t kSmemLimit = 232448;              // sm_100 per-block opt-in 
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxStages = 3;
 constexpr int kQkChunk = 9;                          // K-steps of QK per issue burst
+// An FP8 page lands in its own stage and is widened there: its codes as 8 tiles of 64 rows
+// x 64 bytes at [32, 64) KB (tile c = latent dims [64 c, 64 c + 64)), its scales as 64 rows
+// x 16 bytes at [31, 32) KB, its rope dims (bf16) already in the rope tile at [64, 72) KB.
+// The widened tile c takes [8 c, 8 c + 8) KB. 41,984 bytes land per page, the row format's.
+constexpr uint32_t kF8CodeOff = 32 * 1024;
+constexpr uint32_t kF8ScaleOff = 31 * 1024;
+constexpr uint32_t kF8PageTx = 8 * 64 * 64 + 64 * 16 + kBoxBytes;
 
 // Layout for kN padded query rows. TMEM columns: O^T [0, 4 kN), kSBufs score buffers of 64,
 // then Q's first dims as bf16 pairs. Shared memory (from a 1 KB aligned base): Q's
@@ -82,16 +89,9 @@ struct Cfg {
     static constexpr uint32_t kOffP = kOffQs + kQsChunks * kARows * 128;
     static constexpr uint32_t kOffStage = kOffP + kTileBytes;
     static constexpr uint32_t kMiscBytes = 4096;
-    // FP8 cache: a page's codes and scales (64 rows x 528 bytes) land in one of two staging
-    // buffers and are widened into a bf16 stage; the rope dims land in the stage directly
-    static constexpr uint32_t kF8RowBytes = 528;
-    static constexpr uint32_t kF8PageBytes = 64 * kF8RowBytes;          // 33,792 (33 KB)
-    static constexpr int kF8Stages = kF8 ? 2 : 0;
-    static constexpr int kStagesFit =
-        (int)((kSmemLimit - 1024 - kMiscBytes - kOffStage - kF8Stages * kF8PageBytes) / kStageBytes);
-    static constexpr int kStages = kF8 ? 2 : (kStagesFit > kMaxStages ? kMaxStages : kStagesFit);
-    static constexpr uint32_t kOffF8 = kOffStage + kStages * kStageBytes;
-    static constexpr uint32_t kOffMisc = kOffF8 + kF8Stages * kF8PageBytes;
+    static constexpr int kStagesFit = (int)((kSmemLimit - 1024 - kMiscBytes - kOffStage) / kStageBytes);
+    static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
+    static constexpr uint32_t kOffMisc = kOffStage + kStages * kStageBytes;
     static constexpr uint32_t kSmemAlloc = kOffMisc + kMiscBytes + 1024;     // + base alignment
     static constexpr uint32_t kQSlotBytes = kN * 9 * 128;                    // the q rows' box
     static_assert(kN == 16 || kN == 32 || kN == 64, "kN must be 16, 32 or 64");
@@ -113,9 +113,8 @@ enum : uint32_t {
     kBarEpi = kBarDecide + 1,            // the item's partial row sums / 1/l posted (2 per item)
     kBarDrain = kBarEpi + 1,             // the MMA issuer's last commit
     kBarStall = kBarDrain + 1,           // never completes (the timeout test hook waits on it)
-    kBarF8Full = kBarStall + 1,          // [2] FP8 cache: a staging buffer's copy landed
-    kBarF8Free = kBarF8Full + 2,         // [2] FP8 cache: a staging buffer was widened (4 warps)
-    kBarDqFull = kBarF8Free + 2,         // [kMaxStages] FP8 cache: a stage's page widened (4 warps)
+    kBarWiden = kBarStall + 1,           // FP8 cache: the row group's syncs inside a widening
+    kBarDqFull = kBarWiden + 1,          // [kMaxStages] FP8 cache: a stage's page widened (4 warps)
     kNumBars = kBarDqFull + kMaxStages
 };
 // misc area: barriers [0, 256), tmem base at 256, abort flag at 260; partial maxima
@@ -131,7 +130,6 @@ struct Smem {
     uint64_t wait_limit;                 // ns a wait may last before the kernel gives up
     __device__ uint32_t bar(uint32_t i) const { return base_u32 + C::kOffMisc + 8 * i; }
     __device__ uint32_t stage(uint32_t s) const { return base_u32 + C::kOffStage + s * kStageBytes; }
-    __device__ uint32_t f8buf(uint32_t f) const { return base_u32 + C::kOffF8 + f * C::kF8PageBytes; }
     __device__ uint32_t* tmem_slot() const { return reinterpret_cast<uint32_t*>(base + C::kOffMisc + 256); }
     __device__ volatile int* abort_flag() const {
         return reinterpret_cast<volatile int*>(base + C::kOffMisc + 260);
@@ -195,9 +193,12 @@ __device__ __forceinline__ void warp_arrive(uint32_t bar) {
 
 // ------------------------------------------------------------------ producer (warp 4)
 // Ring slot g uses stage g % kStages; its fill number g / kStages sets the parities.
+// tm_page is the bf16 pool's page map, or for an FP8 cache its codes map; tm_scales and
+// tm_rope are the FP8 cache's scale and rope maps (unused for bf16).
 template <class C>
 __device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<C>& sh,
-                                             const CUtensorMap* tm_page, const CUtensorMap* tm_q) {
+                                             const CUtensorMap* tm_page, const CUtensorMap* tm_scales,
+                                             const CUtensorMap* tm_rope, const CUtensorMap* tm_q) {
     constexpr int kN = C::kN;
     if (g_mla_debug_stall) {
         // test hook: wait on a barrier nothing completes, before any copy is issued, so
@@ -226,8 +227,16 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<C
             if (!(ok = acquire(g))) break;
             const uint32_t s = g % C::kStages;
             const int row = page_row(p, it.b, k, it.k_hi);
-            ptx::mbar_arrive_expect_tx(sh.bar(kBarFull + s), kStageBytes);
-            ptx::tma_load_3d(sh.stage(s), tm_page, sh.bar(kBarFull + s), 0, row, 0);
+            if constexpr (C::kF8) {
+                const uint32_t st = sh.stage(s), bar = sh.bar(kBarFull + s);
+                ptx::mbar_arrive_expect_tx(bar, kF8PageTx);
+                ptx::tma_load_3d(st + kF8CodeOff, tm_page, bar, 0, row, 0);
+                ptx::tma_load_2d(st + kF8ScaleOff, tm_scales, bar, 0, row);
+                ptx::tma_load_2d(st + 8 * kBoxBytes, tm_rope, bar, 0, row);
+            } else {
+                ptx::mbar_arrive_expect_tx(sh.bar(kBarFull + s), kStageBytes);
+                ptx::tma_load_3d(sh.stage(s), tm_page, sh.bar(kBarFull + s), 0, row, 0);
+            }
             ++g;
             if (k + 1 < it.k_hi) {                   // warm L2 for the next page
                 const int pid = p.block_table[(size_t)it.b * p.max_blocks + k + 1];
@@ -238,75 +247,6 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<C
     // every copy issued must land before the CTA may finish
     const uint32_t first = g > (uint32_t)C::kStages ? g - C::kStages : 0u;
     for (uint32_t gg = first; gg < g; ++gg)
-        drain_wait(sh, sh.bar(kBarFull + gg % C::kStages), (gg / C::kStages) & 1u, 0x42u);
-}
-
-// FP8 cache: two cursors over the same items. Cursor A streams each page's codes and
-// scales (box {16 bytes, 33 units, 64 rows}: 528 bytes per row) into the two staging
-// buffers, as far ahead as they free; cursor B fills the bf16 ring in slot order: each
-// item's q rows, then per page its rope dims (box {64, 64 rows} of the bf16 view of the
-// rows, 128-byte swizzle) straight into the stage's rope tile.
-template <class C>
-__device__ __forceinline__ void run_producer_f8(const DecodeParams& p, const Smem<C>& sh,
-                                                const CUtensorMap* tm_codes, const CUtensorMap* tm_rope,
-                                                const CUtensorMap* tm_q) {
-    if (g_mla_debug_stall) {
-        wait_bar(sh, sh.bar(kBarStall), 0, 0x40u);
-        return;
-    }
-    ItemIter ia(p, (int)blockIdx.x, (int)gridDim.x), ib(p, (int)blockIdx.x, (int)gridDim.x);
-    Item a, b;
-    bool have_a = ia.next(a), have_b = ib.next(b);
-    int ka = have_a ? a.k_lo : 0;          // next page of cursor A
-    int kb = -1;                           // next of cursor B: -1 the q slot, else a page
-    uint32_t fa = 0, g = 0;                // staging fills and ring slots issued
-    uint64_t t0 = 0;
-    uint32_t idle = 0;
-    for (;;) {
-        const bool a_ready = have_a && (fa < (uint32_t)C::kF8Stages ||
-            ptx::mbar_test_wait(sh.bar(kBarF8Free + fa % C::kF8Stages), ((fa / C::kF8Stages) - 1u) & 1u));
-        const bool b_ready = have_b && (g < (uint32_t)C::kStages ||
-            ptx::mbar_test_wait(sh.bar(kBarFree + g % C::kStages), ((g / C::kStages) - 1u) & 1u));
-        if (a_ready) {
-            const uint32_t f = fa % C::kF8Stages;
-            ptx::mbar_arrive_expect_tx(sh.bar(kBarF8Full + f), C::kF8PageBytes);
-            ptx::tma_load_3d(sh.f8buf(f), tm_codes, sh.bar(kBarF8Full + f), 0, 0,
-                             page_row(p, a.b, ka, a.k_hi));
-            ++fa;
-            if (++ka >= a.k_hi) { have_a = ia.next(a); ka = have_a ? a.k_lo : 0; }
-            idle = 0;
-        } else if (b_ready) {
-            const uint32_t st = g % C::kStages;
-            if (kb < 0) {
-                ptx::mbar_arrive_expect_tx(sh.bar(kBarFull + st), C::kQSlotBytes);
-                ptx::tma_load_3d(sh.stage(st), tm_q, sh.bar(kBarFull + st), 0,
-                                 b.b * p.rows + b.t * kTileRows, 0);
-                kb = b.k_lo;
-            } else {
-                ptx::mbar_arrive_expect_tx(sh.bar(kBarFull + st), kBoxBytes);
-                ptx::tma_load_2d(sh.stage(st) + 8 * kBoxBytes, tm_rope, sh.bar(kBarFull + st), 0,
-                                 page_row(p, b.b, kb, b.k_hi));
-                if (++kb >= b.k_hi) { have_b = ib.next(b); kb = -1; }
-            }
-            ++g;
-            idle = 0;
-        } else if (!have_a && !have_b) {
-            break;
-        } else if ((++idle & 1023u) == 0) {
-            if (*sh.abort_flag()) break;
-            const uint64_t now = ptx::globaltimer();
-            if (idle == 1024u) t0 = now;
-            else if (now - t0 > sh.wait_limit) {
-                *sh.abort_flag() = 1;
-                record_error(kErrTimeout, 0x43u);
-                break;
-            }
-        }
-    }
-    // every copy issued must land before the CTA may finish
-    for (uint32_t ff = fa > (uint32_t)C::kF8Stages ? fa - C::kF8Stages : 0u; ff < fa; ++ff)
-        drain_wait(sh, sh.bar(kBarF8Full + ff % C::kF8Stages), (ff / C::kF8Stages) & 1u, 0x44u);
-    for (uint32_t gg = g > (uint32_t)C::kStages ? g - C::kStages : 0u; gg < g; ++gg)
         drain_wait(sh, sh.bar(kBarFull + gg % C::kStages), (gg / C::kStages) & 1u, 0x42u);
 }
 
@@ -518,55 +458,82 @@ __device__ __forceinline__ void move_q(const Smem<C>& sh, const RowCtx<C>& c, ui
     ptx::tc_fence_before();
 }
 
-// FP8 cache: widens a page from staging buffer fidx % 2 into the stage of ring slot g, as
-// the 9-tile swizzled bf16 layout QK and PV read (the rope tile arrives by TMA). Thread t
-// takes token t / 2, dims [256 (t % 2), +256): the scales of its two 128-dim groups, and
-// 256 codes, each read back as the format defines it: E4M3 -> f16 (exact), times the
-// scale in fp32, rounded to bf16 (both nearest-even). Rows past the sequence end are
+// Row-group sync inside a widening: every warp arrives, every warp waits (bounded).
+template <class C>
+__device__ __forceinline__ bool widen_sync(const Smem<C>& sh, uint32_t& n_syncs) {
+    warp_arrive(sh.bar(kBarWiden));
+    return warp_wait_bar(sh, sh.bar(kBarWiden), (n_syncs++) & 1u, 0x5au);
+}
+
+// 32 codes of one row (two 16-byte words) to bf16, as the format reads them back: E4M3 ->
+// f16 (exact), times the group scale in fp32, rounded to bf16 (both nearest-even); stored
+// as the row's 16-byte units 4 half .. 4 half + 3 of its 128-byte-swizzled tile row.
+__device__ __forceinline__ void widen32(uint32_t tile_row, int row, int half, float sc,
+                                        const uint4 (&w)[2], bool live) {
+    const uint32_t ws[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+    uint32_t o[16];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t lo = ptx::e4m3x2_to_f16x2((uint16_t)(ws[k] & 0xffffu));
+        const uint32_t hi = ptx::e4m3x2_to_f16x2((uint16_t)(ws[k] >> 16));
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+        const __nv_bfloat162 r0 = __floats2bfloat162_rn(__fmul_rn(a.x, sc), __fmul_rn(a.y, sc));
+        const __nv_bfloat162 r1 = __floats2bfloat162_rn(__fmul_rn(b.x, sc), __fmul_rn(b.y, sc));
+        o[2 * k] = live ? *reinterpret_cast<const uint32_t*>(&r0) : 0u;
+        o[2 * k + 1] = live ? *reinterpret_cast<const uint32_t*>(&r1) : 0u;
+    }
+    const uint32_t sw = (uint32_t)(row & 7);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        ptx::st_shared_v4(tile_row + ((((uint32_t)(4 * half + u)) ^ sw) * 16), o[4 * u], o[4 * u + 1],
+                          o[4 * u + 2], o[4 * u + 3]);
+}
+
+// FP8 cache: widens the page in the stage of ring slot g in place, into the 9-tile
+// swizzled bf16 layout QK and PV read (the rope tile arrived by TMA). Thread t takes row
+// t / 2 and the 32 dims [32 (t % 2), +32) of each 64-dim tile. Widened tiles 4-7 overwrite
+// codes, so the tiles go in order and the row group syncs where an output meets codes
+// not yet read: after the scales are read (tile 3 covers them), after tiles 0-3 (tiles 4
+// and 5 cover codes 0-3), after tiles 4-5 (tile 6 covers codes 4-5), and before tile 7
+// (it covers codes 6-7; its own codes wait in registers). Rows past the sequence end are
 // written as zeros (their codes may be anything, NaN included).
 template <class C>
-__device__ __forceinline__ bool dequant(const Smem<C>& sh, const RowCtx<C>& c, const Item& it,
-                                        int page, uint32_t g, uint32_t fidx) {
-    const uint32_t f = fidx % C::kF8Stages, s = g % C::kStages;
-    if (!warp_wait_bar(sh, sh.bar(kBarF8Full + f), (fidx / C::kF8Stages) & 1u, 0x58u)) return false;
-    if (g >= (uint32_t)C::kStages &&
-        !warp_wait_bar(sh, sh.bar(kBarFree + s), ((g / C::kStages) - 1u) & 1u, 0x59u))
-        return false;
+__device__ __forceinline__ bool widen(const Smem<C>& sh, const RowCtx<C>& c, const Item& it,
+                                      int page, uint32_t g, uint32_t& n_syncs) {
+    const uint32_t s = g % C::kStages;
+    if (!warp_wait_bar(sh, sh.bar(kBarFull + s), (g / C::kStages) & 1u, 0x58u)) return false;
     const int row = c.tid >> 1, half = c.tid & 1;
     const bool live = page * kBlock + row < it.L;
-    const uint32_t src = sh.f8buf(f) + (uint32_t)row * C::kF8RowBytes;
-    const uint32_t dst = sh.stage(s) + (uint32_t)row * 128;
-    const uint4 scv = ptx::ld_shared_v4(src + 512);            // the row's four group scales
-    const float sc0 = __uint_as_float(half ? scv.z : scv.x);
-    const float sc1 = __uint_as_float(half ? scv.w : scv.y);
+    const uint32_t st = sh.stage(s);
+    const uint4 scv = ptx::ld_shared_v4(st + kF8ScaleOff + (uint32_t)row * 16);
+    const float sc[4] = {__uint_as_float(scv.x), __uint_as_float(scv.y), __uint_as_float(scv.z),
+                         __uint_as_float(scv.w)};
+    auto codes = [&](int ch, uint4 (&w)[2]) {
+        const uint32_t a = st + kF8CodeOff + (uint32_t)ch * 4096 + (uint32_t)row * 64 + (uint32_t)half * 32;
+        w[0] = ptx::ld_shared_v4(a);
+        w[1] = ptx::ld_shared_v4(a + 16);
+    };
+    auto tile = [&](int ch, const uint4 (&w)[2]) {
+        widen32(st + (uint32_t)ch * kBoxBytes + (uint32_t)row * 128, row, half, sc[ch >> 1], w, live);
+    };
+    if (!widen_sync(sh, n_syncs)) return false;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {                           // tile 4 half + cc: 64 dims
-        const float sc = cc < 2 ? sc0 : sc1;
-        const uint32_t tile = dst + (uint32_t)(4 * half + cc) * kBoxBytes;
+    for (int ch = 0; ch < 4; ++ch) { uint4 w[2]; codes(ch, w); tile(ch, w); }
+    if (!widen_sync(sh, n_syncs)) return false;
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {                          // 16 codes -> units 2h, 2h+1
-            const uint4 w = ptx::ld_shared_v4(src + (uint32_t)(half * 256 + cc * 64 + h * 16));
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-            uint32_t o[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t lo = ptx::e4m3x2_to_f16x2((uint16_t)(ws[k] & 0xffffu));
-                const uint32_t hi = ptx::e4m3x2_to_f16x2((uint16_t)(ws[k] >> 16));
-                const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
-                const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-                const __nv_bfloat162 r0 = __floats2bfloat162_rn(__fmul_rn(a.x, sc), __fmul_rn(a.y, sc));
-                const __nv_bfloat162 r1 = __floats2bfloat162_rn(__fmul_rn(b.x, sc), __fmul_rn(b.y, sc));
-                o[2 * k] = live ? *reinterpret_cast<const uint32_t*>(&r0) : 0u;
-                o[2 * k + 1] = live ? *reinterpret_cast<const uint32_t*>(&r1) : 0u;
-            }
-            const uint32_t sw = (uint32_t)(row & 7);
-            ptx::st_shared_v4(tile + (((uint32_t)(2 * h) ^ sw) * 16), o[0], o[1], o[2], o[3]);
-            ptx::st_shared_v4(tile + (((uint32_t)(2 * h + 1) ^ sw) * 16), o[4], o[5], o[6], o[7]);
-        }
+    for (int ch = 4; ch < 6; ++ch) { uint4 w[2]; codes(ch, w); tile(ch, w); }
+    if (!widen_sync(sh, n_syncs)) return false;
+    {
+        uint4 w6[2], w7[2];
+        codes(6, w6);
+        tile(6, w6);
+        codes(7, w7);
+        if (!widen_sync(sh, n_syncs)) return false;
+        tile(7, w7);
     }
     ptx::fence_proxy_async_smem();           // the widened tiles visible to the MMA
     warp_arrive(sh.bar(kBarDqFull + s));
-    warp_arrive(sh.bar(kBarF8Free + f));
     return true;
 }
 
@@ -795,6 +762,7 @@ __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<C>& s
     ItemIter iter(p, (int)blockIdx.x, (int)gridDim.x);
     Item it, prev;
     uint32_t g = 0, gs = 0, items = 0;
+    uint32_t n_syncs = 0;                  // FP8: widening syncs so far (their parities)
     Track<C> tr;
     float l_sum = 0.f, l_rnd = 0.f;
     float prev_m = -INFINITY, prev_l = 0.f, prev_r = 0.f;
@@ -822,11 +790,11 @@ __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<C>& s
         // FP8 cache: widen the item's first page now and page j + 1 before the softmax of
         // page j, so QK of the next page finds its operands ready
         if constexpr (C::kF8) {
-            if (!dequant(sh, c, it, it.k_lo, g, gs)) return;
+            if (!widen(sh, c, it, it.k_lo, g, n_syncs)) return;
         }
         for (uint32_t j = 0; j < n; ++j) {
             if constexpr (C::kF8) {
-                if (j + 1 < n && !dequant(sh, c, it, it.k_lo + (int)j + 1, g + j + 1, gs + j + 1)) return;
+                if (j + 1 < n && !widen(sh, c, it, it.k_lo + (int)j + 1, g + j + 1, n_syncs)) return;
             }
             if (!row_step(p, sh, c, it, n_vis, j, gs + j, (g + j) % C::kStages, tr, l_sum, l_rnd))
                 return;
@@ -843,12 +811,13 @@ __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<C>& s
     if (have_prev) epilogue(p, sh, c, prev, prev_m, prev_l, prev_r, gs - 1, items - 1);
 }
 
-// tm_page: the bf16 pool's pages, or for an FP8 cache its rows' codes and scales;
-// tm_rope: FP8 cache only, the rope dims of its rows as bf16 (unused otherwise).
+// tm_page: the bf16 pool's pages, or for an FP8 cache its rows' codes; tm_scales and
+// tm_rope: FP8 cache only, its rows' scales and their rope dims as bf16 (unused otherwise).
 template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
-              const __grid_constant__ CUtensorMap tm_rope, const __grid_constant__ CUtensorMap tm_q) {
+              const __grid_constant__ CUtensorMap tm_scales, const __grid_constant__ CUtensorMap tm_rope,
+              const __grid_constant__ CUtensorMap tm_q) {
     constexpr int kN = C::kN;
     extern __shared__ uint8_t smem_raw[];
     Smem<C> sh;
@@ -876,16 +845,16 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
         ptx::mbar_init(sh.bar(kBarEpi), 4);
         ptx::mbar_init(sh.bar(kBarDrain), 1);
         ptx::mbar_init(sh.bar(kBarStall), 1);
-        for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(sh.bar(kBarF8Full + i), 1);
-            ptx::mbar_init(sh.bar(kBarF8Free + i), 4);
-        }
+        ptx::mbar_init(sh.bar(kBarWiden), 4);
         for (int i = 0; i < kMaxStages; ++i) ptx::mbar_init(sh.bar(kBarDqFull + i), 4);
         *sh.abort_flag() = 0;
         ptx::fence_mbarrier_init_cluster();
         ptx::prefetch_tensormap(&tm_page);
         ptx::prefetch_tensormap(&tm_q);
-        if (C::kF8) ptx::prefetch_tensormap(&tm_rope);
+        if (C::kF8) {
+            ptx::prefetch_tensormap(&tm_scales);
+            ptx::prefetch_tensormap(&tm_rope);
+        }
     }
     if (warp == kWarpMma) {
         ptx::tmem_alloc(ptx::smem_u32(sh.tmem_slot()), kTmemCols);
@@ -899,10 +868,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
     if (warp < 4) {
         run_rows<C>(p, sh, tmem);
     } else if (warp == kWarpProducer) {
-        if (lane == 0) {
-            if constexpr (C::kF8) run_producer_f8<C>(p, sh, &tm_page, &tm_rope, &tm_q);
-            else run_producer<C>(p, sh, &tm_page, &tm_q);
-        }
+        if (lane == 0) run_producer<C>(p, sh, &tm_page, &tm_scales, &tm_rope, &tm_q);
     } else if (warp == kWarpMma) {
         if (lane == 0) run_mma<C>(p, sh, tmem);
     }

@@ -45,9 +45,9 @@ bool shape_ok(int batch, int h_q, int s_q) {
 // above it the 2-CTA kernel (decode_pair.cuh) splits 128-row tiles over two SMs.
 bool use_solo(int h_q, int s_q) { return h_q * s_q <= kSoloMaxRows; }
 
-// Query rows per sequence the FP8-cache decode takes: its two 33 KB staging buffers fit
-// beside two bf16 stages only for the 1-CTA kernel's 16- and 32-row layouts.
-constexpr int kFp8MaxRows = 32;
+// Query rows per sequence the FP8-cache decode takes: the 1-CTA kernel's (each page is
+// widened in its own stage, so every 1-CTA layout carries it).
+constexpr int kFp8MaxRows = kSoloMaxRows;
 
 // Work units a schedule for num_sms SMs may use, before the device cap: one per SM for
 // the 1-CTA kernel, one per SM pair for the 2-CTA kernel.
@@ -331,26 +331,39 @@ mla_status launch_solo(const DecodeParams& p, const void* q, const void* kcache,
     if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
         !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
         return MLA_ERR_CUDA;
-    solo::decode_kernel<C><<<ctas, solo::kThreads, C::kSmemAlloc, s>>>(p, tm_page, tm_page, tm_q);
+    solo::decode_kernel<C><<<ctas, solo::kThreads, C::kSmemAlloc, s>>>(p, tm_page, tm_page, tm_page, tm_q);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// FP8 cache ([num_blocks][64][656] bytes, rows of MLA_FP8_ROW_BYTES): the rows' codes and
-// scales as a 3-D byte view {16 bytes, 41 units of 16 bytes, rows} with box {16, 33, 64}
-// (a page's 64 rows x 528 bytes, dense), and their rope dims as a 2-D bf16 view {64
-// elements, rows} starting 528 bytes into the pool, row stride 656 bytes, box {64, 64},
-// 128-byte swizzle (one swizzled tile, as the bf16 pool's rope chunk lands).
-bool make_f8_maps(CUtensorMap* codes, CUtensorMap* rope, const void* kc8, int num_blocks) {
+// FP8 cache ([num_blocks][64][656] bytes, rows of MLA_FP8_ROW_BYTES), three views a page
+// lands through: the codes as a 3-D byte view {64 bytes, rows, 8 chunks} with strides {656,
+// 64} and box {64, 64, 8}, so a page's 512 codes per row arrive chunk by chunk (64 rows x 64
+// bytes per chunk); the scales as a 2-D byte view {16, rows} starting 512 bytes into the
+// pool, box {16, 64}; the rope dims as a 2-D bf16 view {64, rows} starting 528 bytes in,
+// box {64, 64}, 128-byte swizzle (one swizzled tile, as the bf16 pool's rope chunk lands).
+bool make_f8_maps(CUtensorMap* codes, CUtensorMap* scales, CUtensorMap* rope, const void* kc8,
+                  int num_blocks) {
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return false;
     const cuuint64_t rows = (cuuint64_t)num_blocks * kBlock;
+    char* pool = const_cast<char*>(static_cast<const char*>(kc8));
     {
-        const cuuint64_t dims[3] = {16, MLA_FP8_ROW_BYTES / 16, rows};
-        const cuuint64_t strides[2] = {16, MLA_FP8_ROW_BYTES};
-        const cuuint32_t box[3] = {16, 33, (cuuint32_t)kBlock};
+        const cuuint64_t dims[3] = {64, rows, 8};
+        const cuuint64_t strides[2] = {MLA_FP8_ROW_BYTES, 64};
+        const cuuint32_t box[3] = {64, (cuuint32_t)kBlock, 8};
         const cuuint32_t estr[3] = {1, 1, 1};
-        if (fn(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(kc8), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+        if (fn(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, pool, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    {
+        const cuuint64_t dims[2] = {16, rows};
+        const cuuint64_t strides[1] = {MLA_FP8_ROW_BYTES};
+        const cuuint32_t box[2] = {16, (cuuint32_t)kBlock};
+        const cuuint32_t estr[2] = {1, 1};
+        if (fn(scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, pool + 512, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
     }
@@ -359,8 +372,7 @@ bool make_f8_maps(CUtensorMap* codes, CUtensorMap* rope, const void* kc8, int nu
         const cuuint64_t strides[1] = {MLA_FP8_ROW_BYTES};
         const cuuint32_t box[2] = {64, (cuuint32_t)kBlock};
         const cuuint32_t estr[2] = {1, 1};
-        void* base = const_cast<char*>(static_cast<const char*>(kc8)) + 528;
-        if (fn(rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+        if (fn(rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool + 528, dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return false;
@@ -373,11 +385,12 @@ mla_status launch_solo_f8(const DecodeParams& p, const void* q, const void* kc8,
                           int ctas, int dev, cudaStream_t s) {
     using C = solo::Cfg<kN, true>;
     if (!prepare_solo_kernel<C>(dev)) return MLA_ERR_CUDA;
-    CUtensorMap tm_codes, tm_rope, tm_q;
-    if (!make_f8_maps(&tm_codes, &tm_rope, kc8, num_blocks) ||
+    CUtensorMap tm_codes, tm_scales, tm_rope, tm_q;
+    if (!make_f8_maps(&tm_codes, &tm_scales, &tm_rope, kc8, num_blocks) ||
         !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
         return MLA_ERR_CUDA;
-    solo::decode_kernel<C><<<ctas, solo::kThreads, C::kSmemAlloc, s>>>(p, tm_codes, tm_rope, tm_q);
+    solo::decode_kernel<C><<<ctas, solo::kThreads, C::kSmemAlloc, s>>>(p, tm_codes, tm_scales, tm_rope,
+                                                                       tm_q);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -616,7 +629,8 @@ mla_status mla_decode_fwd_fp8(const uint16_t* q, const uint8_t* kcache_fp8, int 
     if (ctas < 1) return MLA_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
     st = p.rows <= 16 ? launch_solo_f8<16>(p, q, kcache_fp8, num_blocks, ctas, dev, s)
-                      : launch_solo_f8<32>(p, q, kcache_fp8, num_blocks, ctas, dev, s);
+       : p.rows <= 32 ? launch_solo_f8<32>(p, q, kcache_fp8, num_blocks, ctas, dev, s)
+                      : launch_solo_f8<64>(p, q, kcache_fp8, num_blocks, ctas, dev, s);
     if (st != MLA_OK) return st;
     return launch_combine(p, s);
 }

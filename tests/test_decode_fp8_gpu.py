@@ -64,6 +64,9 @@ SMALL = [
     ([258, 3, 1, 0, 64], 3, 7, True),
     ([129, 5], 1, 1, False),
     ([1500, 333], 2, 8, True),
+    ([300, 70, 1], 1, 64, False),
+    ([900, 129], 2, 32, True),
+    ([65, 640], 4, 13, True),
 ]
 
 
@@ -113,9 +116,9 @@ def test_block_permutation_is_bit_exact():
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
 
 
-def test_more_than_32_rows_is_rejected_before_launch():
+def test_more_than_64_rows_is_rejected_before_launch():
     mla = _mla()
-    x = wl.make_paged_inputs([100], 1, 64, seed=6)
+    x = wl.make_paged_inputs([100], 1, 65, seed=6)
     kc8 = f8.quantize_cache(x.kcache)
     with pytest.raises(mla.MlaError) as e:
         run_fp8(x, kc8)
