@@ -117,8 +117,14 @@ int mla_num_work_units(int num_sms, int h_q, int s_q);
  *               single unit and so no splits.
  *   metadata    device int32 [mla_metadata_ints(num_sms)], written:
  *               [0..7]   header {num_units, tiles, batch, h_q, s_q, unit_cost,
- *                        item_overhead, 0}: a work sequence costs its pages plus
- *                        item_overhead (3 for the 2-CTA kernel, 1 for the 1-CTA kernel)
+ *                        item_overhead, tile_aligned}: a work sequence costs its pages
+ *                        plus item_overhead (3 for the 2-CTA kernel, 1 for the 1-CTA
+ *                        kernel). With tiles > 1 row tiles per sequence and at least
+ *                        `tiles` units (tile_aligned = 1), tile t owns units
+ *                        [floor(t U/tiles), floor((t+1) U/tiles)) and balances the
+ *                        batch's pages over them alone, so the tiles of a sequence
+ *                        stream its pages at the same time and DRAM serves each page
+ *                        once; unit_cost is then the largest of the tiles' costs.
  *               [8u+8..] unit u {v_begin, page_begin, v_end, page_end, chunk_begin,0,0,0}
  *                        (half-open range of (v, page) positions)
  *   num_splits  device int32 [mla_num_splits_len(batch, h_q, s_q)], written: the

@@ -18,6 +18,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 // error recorded since the last read sticks.
 enum ErrorKind : uint32_t { kErrNone = 0, kErrTimeout = 1, kErrBadInput = 2, kErrWorkspace = 3 };
 
+// Combine counters per work sequence in the workspace: one per 8-row group of a tile.
+constexpr int kCombineCounters = 16;
+
 // Everything one decode launch needs. Plain pointers; layouts as in include/mla.h.
 struct DecodeParams {
     const __nv_bfloat16* q;        // [batch][s_q][h_q][576]
@@ -37,6 +40,12 @@ struct DecodeParams {
     float scale_log2;              // scale * log2(e): scores kept in the log2 domain
     int causal;
 };
+
+// The combine's counters, [max_chunks][kCombineCounters] int32, follow the output
+// partials in the workspace (their end is 256-byte aligned: 256 KB per slot).
+__device__ __forceinline__ int* combine_counters(const DecodeParams& p) {
+    return reinterpret_cast<int*>(p.ws_o + (size_t)p.max_chunks * kTileRows * kHeadDimV);
+}
 
 // Visible tokens of query i (causal decode appends the s_q queries at the end).
 __device__ __forceinline__ int visible_tokens(int L, int s_q, int i, int causal) {

@@ -267,6 +267,12 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Shared
             if (crank == 0) ptx::mbar_arrive_expect_tx(sh.bar(kBarKFull + (gk & 1u)), 2 * kPageBytes);
             const uint32_t st = sh.stage(gk & 1u);
             ptx::tma_load_3d_pair(st, tm_page, kfull_leader + 8 * (gk & 1u), 0, own, 0);
+            // the holder of a split sequence's first chunk clears the combine's counters
+            if (j == 0 && crank == 0 && it.chunk == 0 && it.n_chunks > 1 && it.v < p.max_chunks) {
+                int* cnt = combine_counters(p) + (size_t)it.v * kCombineCounters;
+#pragma unroll 1
+                for (int i = 0; i < kCombineCounters; ++i) cnt[i] = 0;
+            }
             ++gk;
             if (gk == 2)
                 for (int i = 0; i < kPrefetchSteps; ++i) prefetch_next(true);
@@ -685,6 +691,7 @@ __device__ __forceinline__ bool epilogue(const DecodeParams& p, const Shared& sh
             p.ws_lse[(size_t)it.part * kTileRows + tile_row] = lse2;
         }
     }
+
     ptx::tc_fence_before();
     return true;
 }

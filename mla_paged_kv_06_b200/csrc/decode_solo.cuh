@@ -46,10 +46,12 @@
 namespace mla {
 namespace solo {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;                         // bf16 cache: rows, producer, MMA
+constexpr int kThreadsF8 = 320;                       // FP8 cache: + four widening warps
 constexpr int kRowThreads = 128;
 constexpr int kWarpProducer = 4;
 constexpr int kWarpMma = 5;
+constexpr int kWarpWiden = 6;                         // FP8 cache: warps 6-9 widen pages
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kBoxBytes = 64 * 128;             // 64 rows x 64 bf16, 128-byte swizzle
 constexpr uint32_t kStageBytes = 9 * kBoxBytes;      // one page: 64 tokens x 576 dims
@@ -73,6 +75,7 @@ template <int N_, bool F8_ = false>
 struct Cfg {
     static constexpr int kN = N_;
     static constexpr bool kF8 = F8_;                          // FP8 latent cache (656-byte rows)
+    static constexpr int kBlockThreads = kF8 ? kThreadsF8 : kThreads;
     static constexpr int kRowWarps = kN <= 32 ? 1 : 2;        // warps holding one copy of the rows
     static constexpr int kCopies = 4 / kRowWarps;
     static constexpr int kTok = 64 / kCopies;                 // tokens of a page per warp
@@ -222,6 +225,12 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<C
             ptx::tma_load_3d(sh.stage(s), tm_q, sh.bar(kBarFull + s), 0,
                              it.b * p.rows + it.t * kTileRows, 0);
             ++g;
+        }
+        // the holder of a split sequence's first chunk clears the combine's counters
+        if (it.chunk == 0 && it.n_chunks > 1 && it.v < p.max_chunks) {
+            int* cnt = combine_counters(p) + (size_t)it.v * kCombineCounters;
+#pragma unroll 1
+            for (int i = 0; i < kCombineCounters; ++i) cnt[i] = 0;
         }
         for (int k = it.k_lo; k < it.k_hi; ++k) {
             if (!(ok = acquire(g))) break;
@@ -491,19 +500,19 @@ __device__ __forceinline__ void widen32(uint32_t tile_row, int row, int half, fl
 }
 
 // FP8 cache: widens the page in the stage of ring slot g in place, into the 9-tile
-// swizzled bf16 layout QK and PV read (the rope tile arrived by TMA). Thread t takes row
-// t / 2 and the 32 dims [32 (t % 2), +32) of each 64-dim tile. Widened tiles 4-7 overwrite
+// swizzled bf16 layout QK and PV read (the rope tile arrived by TMA). Thread t (of the
+// four widening warps) takes row t / 2 and the 32 dims [32 (t % 2), +32) of each tile. Widened tiles 4-7 overwrite
 // codes, so the tiles go in order and the row group syncs where an output meets codes
 // not yet read: after the scales are read (tile 3 covers them), after tiles 0-3 (tiles 4
 // and 5 cover codes 0-3), after tiles 4-5 (tile 6 covers codes 4-5), and before tile 7
 // (it covers codes 6-7; its own codes wait in registers). Rows past the sequence end are
 // written as zeros (their codes may be anything, NaN included).
 template <class C>
-__device__ __forceinline__ bool widen(const Smem<C>& sh, const RowCtx<C>& c, const Item& it,
-                                      int page, uint32_t g, uint32_t& n_syncs) {
+__device__ __forceinline__ bool widen(const Smem<C>& sh, int tid, const Item& it, int page,
+                                      uint32_t g, uint32_t& n_syncs) {
     const uint32_t s = g % C::kStages;
     if (!warp_wait_bar(sh, sh.bar(kBarFull + s), (g / C::kStages) & 1u, 0x58u)) return false;
-    const int row = c.tid >> 1, half = c.tid & 1;
+    const int row = tid >> 1, half = tid & 1;
     const bool live = page * kBlock + row < it.L;
     const uint32_t st = sh.stage(s);
     const uint4 scv = ptx::ld_shared_v4(st + kF8ScaleOff + (uint32_t)row * 16);
@@ -713,6 +722,7 @@ __device__ __forceinline__ bool epilogue(const DecodeParams& p, const Smem<C>& s
         }
     }
     if (!final_out && !have_ws && c.tid == 0) record_error(kErrWorkspace, (uint32_t)it.v & 0xffffffu);
+
     warp_arrive(sh.bar(kBarEpi));
     if (!warp_wait_bar(sh, sh.bar(kBarEpi), (2 * epi_index + 1) & 1u, 0x56u)) return false;
     if (!warp_wait_bar(sh, sh.bar(kBarPvDone), last_step & 1u, 0x55u)) return false;
@@ -762,7 +772,6 @@ __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<C>& s
     ItemIter iter(p, (int)blockIdx.x, (int)gridDim.x);
     Item it, prev;
     uint32_t g = 0, gs = 0, items = 0;
-    uint32_t n_syncs = 0;                  // FP8: widening syncs so far (their parities)
     Track<C> tr;
     float l_sum = 0.f, l_rnd = 0.f;
     float prev_m = -INFINITY, prev_l = 0.f, prev_r = 0.f;
@@ -787,15 +796,7 @@ __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<C>& s
         l_sum = 0.f;
         l_rnd = 0.f;
         const uint32_t n = (uint32_t)it.pages();
-        // FP8 cache: widen the item's first page now and page j + 1 before the softmax of
-        // page j, so QK of the next page finds its operands ready
-        if constexpr (C::kF8) {
-            if (!widen(sh, c, it, it.k_lo, g, n_syncs)) return;
-        }
         for (uint32_t j = 0; j < n; ++j) {
-            if constexpr (C::kF8) {
-                if (j + 1 < n && !widen(sh, c, it, it.k_lo + (int)j + 1, g + j + 1, n_syncs)) return;
-            }
             if (!row_step(p, sh, c, it, n_vis, j, gs + j, (g + j) % C::kStages, tr, l_sum, l_rnd))
                 return;
         }
@@ -811,10 +812,26 @@ __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<C>& s
     if (have_prev) epilogue(p, sh, c, prev, prev_m, prev_l, prev_r, gs - 1, items - 1);
 }
 
+// FP8 cache, warps 6-9: widen every page of this CTA's items as it lands, in ring order
+// (an item's q slot comes first and is not theirs), so that neither the softmax warps
+// nor the MMA issuer spend time on it.
+template <class C>
+__device__ __forceinline__ void run_widen(const DecodeParams& p, const Smem<C>& sh, int tid) {
+    ItemIter iter(p, (int)blockIdx.x, (int)gridDim.x);
+    Item it;
+    uint32_t g = 0, n_syncs = 0;
+    while (iter.next(it)) {
+        ++g;                                   // the item's q slot
+        const int n = it.pages();
+        for (int j = 0; j < n; ++j, ++g)
+            if (!widen(sh, tid, it, it.k_lo + j, g, n_syncs)) return;
+    }
+}
+
 // tm_page: the bf16 pool's pages, or for an FP8 cache its rows' codes; tm_scales and
 // tm_rope: FP8 cache only, its rows' scales and their rope dims as bf16 (unused otherwise).
 template <class C>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(C::kBlockThreads, 1)
 decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
               const __grid_constant__ CUtensorMap tm_scales, const __grid_constant__ CUtensorMap tm_rope,
               const __grid_constant__ CUtensorMap tm_q) {
@@ -871,6 +888,8 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
         if (lane == 0) run_producer<C>(p, sh, &tm_page, &tm_scales, &tm_rope, &tm_q);
     } else if (warp == kWarpMma) {
         if (lane == 0) run_mma<C>(p, sh, tmem);
+    } else if (C::kF8 && warp >= kWarpWiden) {
+        run_widen<C>(p, sh, (int)threadIdx.x - 32 * kWarpWiden);
     }
     ptx::tc_fence_before();
     __syncthreads();

@@ -41,7 +41,8 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* smem
     return total;
 }
 
-// metadata: header {num_units, tiles, batch, h_q, s_q, unit_cost, overhead, 0} then one
+// metadata: header {num_units, tiles, batch, h_q, s_q, unit_cost, overhead, tile_aligned}
+// then one
 // {v_begin, page_begin, v_end, page_end, chunk_begin, 0, 0, 0} per unit.
 // num_splits holds the cumulative costs C[v] while the units are located, then is
 // overwritten with the chunk prefix.
@@ -92,18 +93,13 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
         s_total = carry;
     }
     __syncthreads();
-    const int64_t total = s_total;
-    const int64_t W = unit_cost(total, num_units);
     auto C = [&](int v) { return (int64_t)Cs[v]; };
+    const int64_t W = header_unit_cost(num_units, tiles, batch, V, C);
 
     // Phase 2: one thread per unit locates its first and one-past-last page.
     for (int u = threadIdx.x; u < num_units; u += blockDim.x) {
-        int vb, kb, ve, ke;
-        locate((int64_t)u * W, C, pages, V, overhead, &vb, &kb);
-        locate((int64_t)(u + 1) * W, C, pages, V, overhead, &ve, &ke);
-        int chunk = 0;
-        if (vb < V && (vb != ve || kb != ke))
-            chunk = u - unit_of(C(vb) + overhead, W);
+        int vb, kb, ve, ke, chunk;
+        unit_range(u, num_units, tiles, batch, V, overhead, C, pages, &vb, &kb, &ve, &ke, &chunk);
         int32_t* m = metadata + kMetaInts * (u + 1);
         m[0] = vb; m[1] = kb; m[2] = ve; m[3] = ke; m[4] = chunk;
         m[5] = 0; m[6] = 0; m[7] = 0;
@@ -112,7 +108,7 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
         metadata[0] = num_units; metadata[1] = tiles; metadata[2] = batch;
         metadata[3] = h_q; metadata[4] = s_q;
         metadata[5] = (int32_t)(W > 0x7fffffffLL ? 0x7fffffff : W);
-        metadata[6] = overhead; metadata[7] = 0;
+        metadata[6] = overhead; metadata[7] = tile_aligned(tiles, num_units) ? 1 : 0;
     }
     __syncthreads();
 
@@ -121,7 +117,7 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
     carry = 0;
     for (int base = 0; base < V; base += blockDim.x) {
         int v = base + threadIdx.x;
-        int n = v < V ? chunks_of(C(v), pages(v), W, overhead) : 0;
+        int n = v < V ? chunks_of_v(v, num_units, tiles, batch, V, overhead, C, pages) : 0;
         int64_t pre;
         int64_t tot = block_exclusive_scan(n, warp_sums, &pre);   // also a barrier
         if (v < V) num_splits[v] = (int32_t)(carry + pre);

@@ -61,9 +61,13 @@ size_t max_chunks_for(int batch, int h_q, int s_q, int num_sms) {
 }
 
 
-constexpr size_t kChunkBytes = (size_t)kTileRows * 4 + (size_t)kTileRows * kHeadDimV * 4;
+// Per partial slot: 128 rows' lse and outputs (fp32), and the combine's counters of one
+// work sequence (there are never more work sequences than slots).
+constexpr size_t kChunkBytes = (size_t)kTileRows * 4 + (size_t)kTileRows * kHeadDimV * 4 +
+                               (size_t)kCombineCounters * 4;
 
-// Partial-slot capacity of a workspace and the byte offset of its output partials.
+// Partial-slot capacity of a workspace and the byte offsets of its output partials and
+// combine counters.
 size_t ws_capacity(size_t bytes) {
     if (bytes < kWsHeader + 2 * kAlign) return 0;
     return (bytes - kWsHeader - 2 * kAlign) / kChunkBytes;
@@ -71,9 +75,12 @@ size_t ws_capacity(size_t bytes) {
 
 size_t ws_o_offset(size_t cap) { return align_up(kWsHeader + cap * kTileRows * 4, kAlign); }
 
+// The combine counters start right after the output partials (combine_counters()).
+size_t ws_cnt_offset(size_t cap) { return ws_o_offset(cap) + cap * kTileRows * kHeadDimV * 4; }
+
 // Workspace bytes that hold `cap` partial slots.
 size_t workspace_bytes_for(size_t cap) {
-    return ws_o_offset(cap) + cap * kTileRows * kHeadDimV * 4 + kAlign;
+    return ws_cnt_offset(cap) + cap * kCombineCounters * 4 + kAlign;
 }
 
 // Opt the split kernel into its shared-memory footprint (once per device).
@@ -317,7 +324,11 @@ void* noalloc_scratch(int dev) {
 mla_status launch_combine(const DecodeParams& p, cudaStream_t s) {
     // one warp per row of a tile; a tile of a sequence with fewer rows needs fewer CTAs
     const int tile_rows = p.rows < kTileRows ? p.rows : kTileRows;
-    dim3 grid(p.batch * p.tiles, (tile_rows + kCombineRowsPerCta - 1) / kCombineRowsPerCta);
+    // slice CTAs for rows of many chunks only where the grid is small: a big grid's
+    // extra CTAs, which exit at once when no row needs them, cost more than they save
+    const int groups = (tile_rows + kCombineRowsPerCta - 1) / kCombineRowsPerCta;
+    const size_t cells = (size_t)p.batch * p.tiles * groups;
+    dim3 grid(p.batch * p.tiles, groups, cells <= (size_t)kSliceGridMax ? kCombineSlices : 1);
     combine_kernel<<<grid, kCombineThreads, 0, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -389,7 +400,7 @@ mla_status launch_solo_f8(const DecodeParams& p, const void* q, const void* kc8,
     if (!make_f8_maps(&tm_codes, &tm_scales, &tm_rope, kc8, num_blocks) ||
         !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
         return MLA_ERR_CUDA;
-    solo::decode_kernel<C><<<ctas, solo::kThreads, C::kSmemAlloc, s>>>(p, tm_codes, tm_scales, tm_rope,
+    solo::decode_kernel<C><<<ctas, C::kBlockThreads, C::kSmemAlloc, s>>>(p, tm_codes, tm_scales, tm_rope,
                                                                        tm_q);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -696,26 +707,23 @@ mla_status mla_plan_host(const int32_t* seqlens_host, int batch, int h_q, int s_
         C[v + 1] = C[v] + overhead + nblk[v];
     }
     if (C[V] > 0x7fffffffLL) return MLA_ERR_UNSUPPORTED;
-    const int64_t W = unit_cost(C[V], num_units);
     auto cost = [&](int v) { return C[v]; };
     auto pages = [&](int v) { return nblk[v]; };
+    const int64_t W = header_unit_cost(num_units, tiles, batch, V, cost);
     for (int u = 0; u < num_units; ++u) {
-        int vb, kb, ve, ke;
-        locate((int64_t)u * W, cost, pages, V, overhead, &vb, &kb);
-        locate((int64_t)(u + 1) * W, cost, pages, V, overhead, &ve, &ke);
-        int chunk = 0;
-        if (vb < V && (vb != ve || kb != ke)) chunk = u - unit_of(C[vb] + overhead, W);
+        int vb, kb, ve, ke, chunk;
+        unit_range(u, num_units, tiles, batch, V, overhead, cost, pages, &vb, &kb, &ve, &ke, &chunk);
         int32_t* m = metadata_host + kMetaInts * (u + 1);
         m[0] = vb; m[1] = kb; m[2] = ve; m[3] = ke; m[4] = chunk;
         m[5] = 0; m[6] = 0; m[7] = 0;
     }
     metadata_host[0] = num_units; metadata_host[1] = tiles; metadata_host[2] = batch;
     metadata_host[3] = h_q; metadata_host[4] = s_q; metadata_host[5] = (int32_t)W;
-    metadata_host[6] = overhead; metadata_host[7] = 0;
+    metadata_host[6] = overhead; metadata_host[7] = tile_aligned(tiles, num_units) ? 1 : 0;
     int32_t acc = 0;
     for (int v = 0; v < V; ++v) {
         num_splits_host[v] = acc;
-        acc += chunks_of(C[v], nblk[v], W, overhead);
+        acc += chunks_of_v(v, num_units, tiles, batch, V, overhead, cost, pages);
     }
     num_splits_host[V] = acc;
     return MLA_OK;

@@ -9,9 +9,16 @@
 // With W = max(ceil(C[V] / units), kMinUnitCost), unit u owns every page whose position lies in
 // [u*W, (u+1)*W). So each unit owns one contiguous run of pages, every page has
 // exactly one owner, and a work sequence whose pages straddle a multiple of W is
-// split there. Tile-major numbering puts tile t of sequence b about units/tiles units
-// after tile t-1 of b, so both tiles stream the same pages at about the same time and
-// the second read hits L2.
+// split there.
+//
+// Tile-aligned cut. With T > 1 row tiles per sequence and at least T units, every tile
+// has the same cost line (the pages are the sequence's), so the line is cut per tile:
+// tile t owns units [floor(t U / T), floor((t+1) U / T)) and cuts its own line of the
+// batch's costs C[0..batch] with W_t = max(ceil(C[batch] / U_t), kMinUnitCost). Where
+// the tiles get equal unit counts, unit u of tile 0 and unit u + U/T of tile 1 own the
+// same pages in the same order and stream them at the same time, so each page comes
+// from DRAM once for all tiles. (On one line the tiles' runs drift apart by up to W
+// pages, and the second read of a page missed L2.)
 #pragma once
 
 #include <stdint.h>
@@ -67,6 +74,42 @@ MLA_HD int chunks_of(int64_t Cv, int nblk, int64_t W, int overhead) {
     return unit_of(p1, W) - unit_of(p0, W) + 1;
 }
 
+MLA_HD bool tile_aligned(int tiles, int units) { return tiles > 1 && units >= tiles; }
+MLA_HD int tile_first_unit(int t, int tiles, int units) {
+    return (int)(((int64_t)t * units) / tiles);
+}
+
+// Where unit u cuts: the line it cuts (its first work sequence v0 and sequence count n,
+// the costs of that line being C[v0 + i] - C[v0]), its index within the line's units and
+// the line's per-unit cost. C(v) is the cumulative cost over all V work sequences.
+struct UnitCut {
+    int v0, n, local;
+    int64_t W;
+};
+
+template <class CostFn>
+MLA_HD UnitCut cut_of_unit(int u, int units, int tiles, int batch, int V, CostFn C) {
+    UnitCut c;
+    if (!tile_aligned(tiles, units)) {
+        c.v0 = 0; c.n = V; c.local = u;
+        c.W = unit_cost(C(V), units);
+        return c;
+    }
+    const int t = (int)((((int64_t)u + 1) * tiles - 1) / units);
+    const int first = tile_first_unit(t, tiles, units);
+    c.v0 = t * batch; c.n = batch; c.local = u - first;
+    c.W = unit_cost(C(batch), tile_first_unit(t + 1, tiles, units) - first);
+    return c;
+}
+
+// Per-unit cost of the line work sequence v lies on.
+template <class CostFn>
+MLA_HD int64_t line_cost_of(int v, int units, int tiles, int batch, int V, CostFn C) {
+    if (!tile_aligned(tiles, units)) return unit_cost(C(V), units);
+    const int t = v / batch;
+    return unit_cost(C(batch), tile_first_unit(t + 1, tiles, units) - tile_first_unit(t, tiles, units));
+}
+
 // Unit range record written into metadata[8 + 8u ..].
 struct UnitRange {
     int v_begin, page_begin, v_end, page_end, chunk_begin;
@@ -91,6 +134,44 @@ MLA_HD void locate(const int64_t target, CostFn C, PagesFn nblk, int V, int over
     int64_t k = target - ((int64_t)C(v) + overhead);
     *v_out = v;
     *k_out = k < 0 ? 0 : (int)k;
+}
+
+// Unit u's run [(vb, kb), (ve, ke)) in (work sequence, page) order, and the chunk index
+// of its first work sequence. C(v) over [0, V] and nblk(v) are the cost line's inputs.
+template <class CostFn, class PagesFn>
+MLA_HD void unit_range(int u, int units, int tiles, int batch, int V, int overhead, CostFn C,
+                       PagesFn nblk, int* vb, int* kb, int* ve, int* ke, int* chunk) {
+    const UnitCut c = cut_of_unit(u, units, tiles, batch, V, C);
+    const int64_t base = C(c.v0);
+    auto Cl = [&](int i) { return (int64_t)C(c.v0 + i) - base; };
+    auto Pl = [&](int i) { return nblk(c.v0 + i); };
+    int b0, k0, b1, k1;
+    locate((int64_t)c.local * c.W, Cl, Pl, c.n, overhead, &b0, &k0);
+    locate((int64_t)(c.local + 1) * c.W, Cl, Pl, c.n, overhead, &b1, &k1);
+    int ch = 0;
+    if (b0 < c.n && (b0 != b1 || k0 != k1)) ch = c.local - unit_of(Cl(b0) + overhead, c.W);
+    *vb = c.v0 + b0; *kb = k0; *ve = c.v0 + b1; *ke = k1; *chunk = ch;
+}
+
+// Chunks work sequence v is split into under the cut above.
+template <class CostFn, class PagesFn>
+MLA_HD int chunks_of_v(int v, int units, int tiles, int batch, int V, int overhead, CostFn C,
+                       PagesFn nblk) {
+    const int v0 = tile_aligned(tiles, units) ? (v / batch) * batch : 0;
+    const int64_t W = line_cost_of(v, units, tiles, batch, V, C);
+    return chunks_of((int64_t)C(v) - (int64_t)C(v0), nblk(v), W, overhead);
+}
+
+// The metadata header's unit cost: the largest per-unit cost of any line.
+template <class CostFn>
+MLA_HD int64_t header_unit_cost(int units, int tiles, int batch, int V, CostFn C) {
+    if (!tile_aligned(tiles, units)) return unit_cost(C(V), units);
+    int64_t w = 0;
+    for (int t = 0; t < tiles; ++t) {
+        const int64_t wt = line_cost_of(t * batch, units, tiles, batch, V, C);
+        w = wt > w ? wt : w;
+    }
+    return w;
 }
 
 }  // namespace mla

@@ -157,13 +157,48 @@ def test_schedule_random_and_balanced():
         overhead = 1 if h_q * s_q <= 64 else 3
         assert int(meta[6]) == overhead
         total = sum(overhead + n for n in nblk)
-        assert W == max(-(-total // U), 4)
+        T = int(meta[1])
+        if T > 1 and U >= T:
+            # tile-aligned: tile t cuts its own line (the batch's costs) over its units
+            assert int(meta[7]) == 1
+            line = total // T
+            units_t = [(t + 1) * U // T - t * U // T for t in range(T)]
+            assert W == max(max(-(-line // n), 4) for n in units_t)
+        else:
+            assert int(meta[7]) == 0
+            assert W == max(-(-total // U), 4)
         # no unit owns more than W pages: the largest unit is within one overhead of ideal
         per_unit = [0] * U
         for v, items in seen.items():
             for (u, _, _) in items:
                 per_unit[u] += 1
         assert max(per_unit) <= W
+
+
+@pytest.mark.parametrize("s_q,U", [(2, 74), (4, 74), (3, 74), (2, 5)])
+def test_tile_aligned_units_of_equal_count_stream_the_same_pages(s_q, U):
+    # Several row tiles: tile t owns units [t U / T, (t+1) U / T) and cuts the batch's
+    # cost line over them alone, so tiles with equal unit counts get the same runs
+    rng = random.Random(s_q * 100 + U)
+    lens = [rng.randint(0, 9000) for _ in range(57)] + [65536, 1, 0]
+    B = len(lens)
+    meta, ns = mla.mla_plan_host(lens, 128, s_q, U)
+    _walk(meta, ns, lens, 128, s_q)
+    T = int(meta[1])
+    assert T == s_q and int(meta[7]) == 1
+    first = [t * U // T for t in range(T + 1)]
+    rec = lambda u: [int(x) for x in meta[8 * (u + 1): 8 * (u + 1) + 5]]
+    for t in range(1, T):
+        if first[t + 1] - first[t] != first[1] - first[0]:
+            continue
+        for i in range(first[1] - first[0]):
+            a, b = rec(first[0] + i), rec(first[t] + i)
+            assert [b[0] - t * B, b[1], b[2] - t * B, b[3], b[4]] == a, (t, i, a, b)
+    # every tile's chunk counts are the same
+    n = np.diff(ns)
+    for t in range(1, T):
+        if first[t + 1] - first[t] == first[1] - first[0]:
+            assert np.array_equal(n[t * B:(t + 1) * B], n[:B])
 
 
 def test_schedule_no_split_with_one_unit():

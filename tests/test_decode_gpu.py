@@ -187,6 +187,28 @@ def test_thirty_thousand_sequences_sharing_a_small_pool():
 FULL = ["uniform", "v3", "spec", "skewed"]
 
 
+@pytest.mark.parametrize("h_q,s_q,num_sms,chunks", [
+    (16, 1, 8, 8), (16, 1, 9, 9), (16, 1, 17, 17), (16, 1, 33, 33), (16, 1, 148, 129),
+    (128, 2, 40, 10), (128, 2, 140, 34),
+])
+def test_rows_merged_from_many_chunks(h_q, s_q, num_sms, chunks):
+    # One long sequence spread over every unit: the combine cuts a row of more than 8
+    # chunks into slices merged by separate CTAs and then merges the slices. Short
+    # sequences beside it keep the one-pass merge.
+    mla = _mla()
+    lens = [40960, 100, 0, 64]
+    x = wl.make_paged_inputs(lens, s_q, h_q, seed=chunks + h_q, causal=s_q > 1,
+                             spare_blocks=2, poison=True)
+    nsm = min(num_sms, mla.default_num_sms())
+    _, ns = mla.mla_plan_host(lens, h_q, s_q, mla.mla_num_work_units(nsm, h_q, s_q))
+    if nsm == num_sms:
+        assert int(ns[1] - ns[0]) == chunks      # the first sequence's chunks (tile 0)
+    out, lse = run(x, num_sms=nsm)
+    compare(out, lse, *oracle_all(x), what=f"{h_q}/{s_q}/{nsm}")
+    out2, lse2 = run(x, num_sms=nsm)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
 @pytest.fixture(scope="module")
 def full_inputs():
     cache = {}
