@@ -34,16 +34,22 @@ namespace mla {
 constexpr int kBlock = 64;
 constexpr int kTileRows = 128;
 // Fixed cost of one work sequence in page units: loading its query tile, refilling the
-// pipeline and its epilogue. Measured on B200: an item boundary of the 2-CTA kernel costs
-// about as much as three and a half pages; one of the 1-CTA kernel (sequences of at most
+// pipeline and its epilogue. Measured on B200 (per-CTA timelines, a least-squares fit of
+// unit time over pages and items): an item boundary of the 2-CTA kernel costs about as
+// much as three and a half pages; one of the 1-CTA kernel (sequences of at most
 // kSoloMaxRows query rows), whose q rows ride in a slot of the page ring and whose
-// epilogue overlaps the next item's first QK, about half a page.
+// epilogue overlaps the next item's first QK, about 0.6 of a page with 16 rows (three
+// stages) but 2.5 pages with 64 rows (two stages, a 72 KB q slot and a 48 KB copy of the
+// q rows into shared memory).
 constexpr int kOverheadPages = 3;
 constexpr int kOverheadPagesSolo = 1;
+constexpr int kOverheadPagesSoloWide = 3;   // 1-CTA kernel, 33-64 query rows
 constexpr int kSoloMaxRows = 64;
 
 MLA_HD int overhead_pages(int h_q, int s_q) {
-    return h_q * s_q <= kSoloMaxRows ? kOverheadPagesSolo : kOverheadPages;
+    const int rows = h_q * s_q;
+    if (rows > kSoloMaxRows) return kOverheadPages;
+    return rows <= 32 ? kOverheadPagesSolo : kOverheadPagesSoloWide;
 }
 constexpr int kMetaInts = 8;
 // Smallest per-unit cost: a split costs a partial tile write and a combine read, so

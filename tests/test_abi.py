@@ -152,9 +152,10 @@ def test_schedule_random_and_balanced():
         meta, ns = mla.mla_plan_host(lens, h_q, s_q, U)
         seen, nblk = _walk(meta, ns, lens, h_q, s_q)
         W = int(meta[5])
-        # fixed cost per work sequence, in pages: 1 for the 1-CTA kernel (at most 64 query
-        # rows per sequence), 3 for the 2-CTA kernel; the header records it
-        overhead = 1 if h_q * s_q <= 64 else 3
+        # fixed cost per work sequence, in pages: 1 for the 1-CTA kernel up to 32 query
+        # rows per sequence, 3 for it with 33-64 rows and for the 2-CTA kernel; the header
+        # records it
+        overhead = 1 if h_q * s_q <= 32 else 3
         assert int(meta[6]) == overhead
         total = sum(overhead + n for n in nblk)
         T = int(meta[1])
