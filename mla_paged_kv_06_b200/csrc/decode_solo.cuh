@@ -47,11 +47,12 @@ namespace mla {
 namespace solo {
 
 constexpr int kThreads = 192;                         // bf16 cache: rows, producer, MMA
-constexpr int kThreadsF8 = 320;                       // FP8 cache: + four widening warps
+constexpr int kWidenWarps = 8;                        // FP8 cache: warps that widen pages
+constexpr int kThreadsF8 = kThreads + 32 * kWidenWarps;
 constexpr int kRowThreads = 128;
 constexpr int kWarpProducer = 4;
 constexpr int kWarpMma = 5;
-constexpr int kWarpWiden = 6;                         // FP8 cache: warps 6-9 widen pages
+constexpr int kWarpWiden = 6;                         // FP8 cache: the first widening warp
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kBoxBytes = 64 * 128;             // 64 rows x 64 bf16, 128-byte swizzle
 constexpr uint32_t kStageBytes = 9 * kBoxBytes;      // one page: 64 tokens x 576 dims
@@ -116,8 +117,8 @@ enum : uint32_t {
     kBarEpi = kBarDecide + 1,            // the item's partial row sums / 1/l posted (2 per item)
     kBarDrain = kBarEpi + 1,             // the MMA issuer's last commit
     kBarStall = kBarDrain + 1,           // never completes (the timeout test hook waits on it)
-    kBarWiden = kBarStall + 1,           // FP8 cache: the row group's syncs inside a widening
-    kBarDqFull = kBarWiden + 1,          // [kMaxStages] FP8 cache: a stage's page widened (4 warps)
+    kBarWiden = kBarStall + 1,           // FP8 cache: the widening warps' syncs inside a page
+    kBarDqFull = kBarWiden + 1,          // [kMaxStages] FP8 cache: a stage's page widened (kWidenWarps arrivals)
     kNumBars = kBarDqFull + kMaxStages
 };
 // misc area: barriers [0, 256), tmem base at 256, abort flag at 260; partial maxima
@@ -474,34 +475,38 @@ __device__ __forceinline__ bool widen_sync(const Smem<C>& sh, uint32_t& n_syncs)
     return warp_wait_bar(sh, sh.bar(kBarWiden), (n_syncs++) & 1u, 0x5au);
 }
 
-// 32 codes of one row (two 16-byte words) to bf16, as the format reads them back: E4M3 ->
-// f16 (exact), times the group scale in fp32, rounded to bf16 (both nearest-even); stored
-// as the row's 16-byte units 4 half .. 4 half + 3 of its 128-byte-swizzled tile row.
-__device__ __forceinline__ void widen32(uint32_t tile_row, int row, int half, float sc,
-                                        const uint4 (&w)[2], bool live) {
-    const uint32_t ws[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
-    uint32_t o[16];
+// 16 kU codes of one row (kU 16-byte words) to bf16, as the format reads them back: E4M3
+// -> f16 (exact), times the group scale in fp32, rounded to bf16 (both nearest-even);
+// stored as the row's 16-byte units 2 kU part .. 2 kU part + 2 kU - 1 of its
+// 128-byte-swizzled tile row.
+template <int kU>
+__device__ __forceinline__ void widen_units(uint32_t tile_row, int row, int part, float sc,
+                                            const uint4 (&w)[kU], bool live) {
+    uint32_t o[8 * kU];
+    const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const uint32_t lo = ptx::e4m3x2_to_f16x2((uint16_t)(ws[k] & 0xffffu));
-        const uint32_t hi = ptx::e4m3x2_to_f16x2((uint16_t)(ws[k] >> 16));
-        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
-        const __nv_bfloat162 r0 = __floats2bfloat162_rn(__fmul_rn(a.x, sc), __fmul_rn(a.y, sc));
-        const __nv_bfloat162 r1 = __floats2bfloat162_rn(__fmul_rn(b.x, sc), __fmul_rn(b.y, sc));
+    for (int k = 0; k < 4 * kU; ++k) {
+        const uint4& wu = w[k >> 2];
+        const uint32_t word = (k & 3) == 0 ? wu.x : (k & 3) == 1 ? wu.y : (k & 3) == 2 ? wu.z : wu.w;
+        const uint32_t lo = ptx::e4m3x2_to_f16x2((uint16_t)(word & 0xffffu));
+        const uint32_t hi = ptx::e4m3x2_to_f16x2((uint16_t)(word >> 16));
+        const float2 a = ptx::mul_f32x2(__half22float2(*reinterpret_cast<const __half2*>(&lo)), sc2);
+        const float2 b = ptx::mul_f32x2(__half22float2(*reinterpret_cast<const __half2*>(&hi)), sc2);
+        const __nv_bfloat162 r0 = __floats2bfloat162_rn(a.x, a.y);
+        const __nv_bfloat162 r1 = __floats2bfloat162_rn(b.x, b.y);
         o[2 * k] = live ? *reinterpret_cast<const uint32_t*>(&r0) : 0u;
         o[2 * k + 1] = live ? *reinterpret_cast<const uint32_t*>(&r1) : 0u;
     }
     const uint32_t sw = (uint32_t)(row & 7);
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-        ptx::st_shared_v4(tile_row + ((((uint32_t)(4 * half + u)) ^ sw) * 16), o[4 * u], o[4 * u + 1],
-                          o[4 * u + 2], o[4 * u + 3]);
+    for (int u = 0; u < 2 * kU; ++u)
+        ptx::st_shared_v4(tile_row + ((((uint32_t)(2 * kU * part + u)) ^ sw) * 16), o[4 * u],
+                          o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
 }
 
 // FP8 cache: widens the page in the stage of ring slot g in place, into the 9-tile
-// swizzled bf16 layout QK and PV read (the rope tile arrived by TMA). Thread t (of the
-// four widening warps) takes row t / 2 and the 32 dims [32 (t % 2), +32) of each tile. Widened tiles 4-7 overwrite
+// swizzled bf16 layout QK and PV read (the rope tile arrived by TMA). The widening warps
+// give each row kWidenWarps / 2 threads, each a contiguous share of each tile's 64 dims. Widened tiles 4-7 overwrite
 // codes, so the tiles go in order and the row group syncs where an output meets codes
 // not yet read: after the scales are read (tile 3 covers them), after tiles 0-3 (tiles 4
 // and 5 cover codes 0-3), after tiles 4-5 (tile 6 covers codes 4-5), and before tile 7
@@ -512,29 +517,33 @@ __device__ __forceinline__ bool widen(const Smem<C>& sh, int tid, const Item& it
                                       uint32_t g, uint32_t& n_syncs) {
     const uint32_t s = g % C::kStages;
     if (!warp_wait_bar(sh, sh.bar(kBarFull + s), (g / C::kStages) & 1u, 0x58u)) return false;
-    const int row = tid >> 1, half = tid & 1;
+    // kParts threads per row, each kU 16-byte words (16 kU codes) of each 64-code chunk
+    constexpr int kParts = kWidenWarps * 32 / kBlock;
+    constexpr int kU = 4 / kParts;
+    static_assert(kParts * kU == 4 && kParts * kBlock == kWidenWarps * 32, "widening layout");
+    const int row = tid / kParts, part = tid % kParts;
     const bool live = page * kBlock + row < it.L;
     const uint32_t st = sh.stage(s);
     const uint4 scv = ptx::ld_shared_v4(st + kF8ScaleOff + (uint32_t)row * 16);
     const float sc[4] = {__uint_as_float(scv.x), __uint_as_float(scv.y), __uint_as_float(scv.z),
                          __uint_as_float(scv.w)};
-    auto codes = [&](int ch, uint4 (&w)[2]) {
-        const uint32_t a = st + kF8CodeOff + (uint32_t)ch * 4096 + (uint32_t)row * 64 + (uint32_t)half * 32;
-        w[0] = ptx::ld_shared_v4(a);
-        w[1] = ptx::ld_shared_v4(a + 16);
+    auto codes = [&](int ch, uint4 (&w)[kU]) {
+        const uint32_t a = st + kF8CodeOff + (uint32_t)ch * 4096 + (uint32_t)row * 64 + (uint32_t)part * 16 * kU;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) w[u] = ptx::ld_shared_v4(a + 16 * u);
     };
-    auto tile = [&](int ch, const uint4 (&w)[2]) {
-        widen32(st + (uint32_t)ch * kBoxBytes + (uint32_t)row * 128, row, half, sc[ch >> 1], w, live);
+    auto tile = [&](int ch, const uint4 (&w)[kU]) {
+        widen_units<kU>(st + (uint32_t)ch * kBoxBytes + (uint32_t)row * 128, row, part, sc[ch >> 1], w, live);
     };
     if (!widen_sync(sh, n_syncs)) return false;
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch) { uint4 w[2]; codes(ch, w); tile(ch, w); }
+    for (int ch = 0; ch < 4; ++ch) { uint4 w[kU]; codes(ch, w); tile(ch, w); }
     if (!widen_sync(sh, n_syncs)) return false;
 #pragma unroll
-    for (int ch = 4; ch < 6; ++ch) { uint4 w[2]; codes(ch, w); tile(ch, w); }
+    for (int ch = 4; ch < 6; ++ch) { uint4 w[kU]; codes(ch, w); tile(ch, w); }
     if (!widen_sync(sh, n_syncs)) return false;
     {
-        uint4 w6[2], w7[2];
+        uint4 w6[kU], w7[kU];
         codes(6, w6);
         tile(6, w6);
         codes(7, w7);
@@ -862,8 +871,8 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
         ptx::mbar_init(sh.bar(kBarEpi), 4);
         ptx::mbar_init(sh.bar(kBarDrain), 1);
         ptx::mbar_init(sh.bar(kBarStall), 1);
-        ptx::mbar_init(sh.bar(kBarWiden), 4);
-        for (int i = 0; i < kMaxStages; ++i) ptx::mbar_init(sh.bar(kBarDqFull + i), 4);
+        ptx::mbar_init(sh.bar(kBarWiden), kWidenWarps);
+        for (int i = 0; i < kMaxStages; ++i) ptx::mbar_init(sh.bar(kBarDqFull + i), kWidenWarps);
         *sh.abort_flag() = 0;
         ptx::fence_mbarrier_init_cluster();
         ptx::prefetch_tensormap(&tm_page);
