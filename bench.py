@@ -299,12 +299,21 @@ def time_split_kv(mla, flush, stream, steps, seed):
                     "timed"}
 
 
+# B200 nominal peaks (HGX HBM3e bandwidth, dense bf16 tensor rate), reported beside the
+# measured ones as the stricter reference
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
 def roofline_fracs(nbytes, nflops, seconds, hbm_peak, tf_peak):
     t_bytes = nbytes / (hbm_peak * 1e9)
     t_flops = nflops / (tf_peak * 1e12)
+    n_bytes = nbytes / (NOMINAL_HBM_GBS * 1e9)
+    n_flops = nflops / (NOMINAL_BF16_TFLOPS * 1e12)
     return {"bound": "hbm" if t_bytes >= t_flops else "tensor",
             "hbm_frac": t_bytes / seconds, "tensor_frac": t_flops / seconds,
-            "roofline_frac": max(t_bytes, t_flops) / seconds}
+            "roofline_frac": max(t_bytes, t_flops) / seconds,
+            "roofline_frac_nominal": max(n_bytes, n_flops) / seconds}
 
 
 def time_config(mla, name, seed, flush, stream, steps, warmup, hbm_peak, tf_peak,
@@ -647,6 +656,8 @@ def main():
             "traffic": traffic,
             "hbm_frac": achieved_gbs / hbm_peak, "tensor_frac": achieved_tf / tf_peak,
             "roofline_frac": max(t_bytes, t_flops) / avg_decode_s,
+            "roofline_frac_nominal": max(nbytes / (NOMINAL_HBM_GBS * 1e9),
+                                         nflops / (NOMINAL_BF16_TFLOPS * 1e12)) / avg_decode_s,
             "algorithmic_bytes": nbytes, "algorithmic_flops": nflops}
 
     value = nbytes * args.steps * world / (total_ms / 1e3) / 1e9
