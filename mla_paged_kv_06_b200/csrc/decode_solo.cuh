@@ -457,10 +457,13 @@ __device__ __forceinline__ void move_q(const Smem<C>& sh, const RowCtx<C>& c, ui
         for (int ch = 0; ch < C::kQsChunks; ++ch) {
             const uint32_t src = st + (C::kQtChunks + ch) * C::kTileBytes + (uint32_t)r * 128;
             const uint32_t dst = sh.base_u32 + C::kOffQs + ch * (C::kARows * 128) + (uint32_t)a * 128;
+            // 16-byte units in an order rotated by row, so that a warp's 32 rows spread
+            // over all banks (the copy keeps each unit in place)
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const uint4 x = ptx::ld_shared_v4(src + u * 16);
-                ptx::st_shared_v4(dst + u * 16, x.x, x.y, x.z, x.w);
+                const uint32_t off = (uint32_t)((u ^ a) & 7) * 16;
+                const uint4 x = ptx::ld_shared_v4(src + off);
+                ptx::st_shared_v4(dst + off, x.x, x.y, x.z, x.w);
             }
         }
     }
