@@ -18,7 +18,7 @@
 //        tile itself, read MN-major from its stage (no copy); P is the B operand, K-major,
 //        one 128-byte row of 64 bf16 probabilities per query row, each warp writing its
 //        token slice. O^T needs 4 kN TMEM columns, which leaves room for Q in TMEM.
-// Per CTA (192 threads):
+// Per CTA (224 threads; 480 over an FP8 cache):
 //   warps 0-3  the row group. Warp w takes copy w / kRowWarps of the rows (token slice
 //              [copy x kTok, +kTok) of every page) and rows (w % kRowWarps) x 32 + lane.
 //              All 128 threads (TMEM lane = latent dim of an O^T block) also do the rare
@@ -28,9 +28,14 @@
 //              q rows (box {64, kN rows, 9 chunks}) and then one slot per page (box {64,
 //              64 rows, 9 chunks}: 9 swizzled 8 KB tiles in one instruction), with the next
 //              page prefetched into L2.
-//   warp 5     TMEM owner and MMA issuer, in the order QK(0) QK(1) PV(0) QK(2) PV(1) ...:
-//              the next page's QK keeps the tensor pipe busy while the row group turns
-//              S(j) into P(j).
+//   warp 5     TMEM owner and QK issuer: each page's QK as soon as its stage landed and
+//              its score buffer was read out, so the next page's QK keeps the tensor pipe
+//              busy while the row group turns S(j) into P(j).
+//   warp 6     PV issuer: PV(j) as soon as P(j) is written. With one thread issuing both,
+//              a P that became ready while the next QK's 36 instructions were being
+//              issued (the issue queue is shallow, so that thread blocks) waited for all
+//              of them, and its stage stayed held that much longer.
+//   warps 7-14 FP8 cache only: widen each page's codes to bf16 in its stage.
 // Scores stay in the log2 domain. A row's reference max is raised only when a score
 // exceeds it by more than kRescaleLog2. Partial maxima of the token slices meet in shared
 // memory once per page; every warp then tracks every row's reference itself, so the
@@ -46,13 +51,14 @@
 namespace mla {
 namespace solo {
 
-constexpr int kThreads = 192;                         // bf16 cache: rows, producer, MMA
+constexpr int kThreads = 224;                         // bf16 cache: rows, producer, QK and PV issuers
 constexpr int kWidenWarps = 8;                        // FP8 cache: warps that widen pages
 constexpr int kThreadsF8 = kThreads + 32 * kWidenWarps;
 constexpr int kRowThreads = 128;
 constexpr int kWarpProducer = 4;
-constexpr int kWarpMma = 5;
-constexpr int kWarpWiden = 6;                         // FP8 cache: the first widening warp
+constexpr int kWarpMma = 5;                           // issues QK (and owns TMEM)
+constexpr int kWarpPv = 6;                            // issues PV
+constexpr int kWarpWiden = 7;                         // FP8 cache: the first widening warp
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kBoxBytes = 64 * 128;             // 64 rows x 64 bf16, 128-byte swizzle
 constexpr uint32_t kStageBytes = 9 * kBoxBytes;      // one page: 64 tokens x 576 dims
@@ -110,13 +116,13 @@ enum : uint32_t {
     kBarQkDone = kBarFree + kMaxStages,  // [2] QK of a step done (score buffer step % kSBufs)
     kBarPvDone = kBarQkDone + 2,         // PV of a step done (one phase per step)
     kBarPReady = kBarPvDone + 1,         // the row group wrote P (4 warp arrivals)
-    kBarSFree = kBarPReady + 1,          // the row group read S out (single buffer only)
-    kBarQReady = kBarSFree + 1,          // the item's q rows are in TMEM and shared memory
+    kBarSFree = kBarPReady + 1,          // [2] the row group read S out of score buffer i
+    kBarQReady = kBarSFree + 2,          // the item's q rows are in TMEM and shared memory
     kBarOFree = kBarQReady + 1,          // the previous item's O^T was read out
     kBarDecide = kBarOFree + 1,          // the step's partial maxima are posted
     kBarEpi = kBarDecide + 1,            // the item's partial row sums / 1/l posted (2 per item)
-    kBarDrain = kBarEpi + 1,             // the MMA issuer's last commit
-    kBarStall = kBarDrain + 1,           // never completes (the timeout test hook waits on it)
+    kBarDrain = kBarEpi + 1,             // [2] the QK and the PV issuer's last commits
+    kBarStall = kBarDrain + 2,           // never completes (the timeout test hook waits on it)
     kBarWiden = kBarStall + 1,           // FP8 cache: the widening warps' syncs inside a page
     kBarDqFull = kBarWiden + 1,          // [kMaxStages] FP8 cache: a stage's page widened (kWidenWarps arrivals)
     kNumBars = kBarDqFull + kMaxStages
@@ -203,7 +209,6 @@ template <class C>
 __device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<C>& sh,
                                              const CUtensorMap* tm_page, const CUtensorMap* tm_scales,
                                              const CUtensorMap* tm_rope, const CUtensorMap* tm_q) {
-    constexpr int kN = C::kN;
     if (g_mla_debug_stall) {
         // test hook: wait on a barrier nothing completes, before any copy is issued, so
         // every role gives up after the limit with nothing in flight
@@ -260,12 +265,11 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<C
         drain_wait(sh, sh.bar(kBarFull + gg % C::kStages), (gg / C::kStages) & 1u, 0x42u);
 }
 
-// ------------------------------------------------------------------ MMA issuer (warp 5)
+// ------------------------------------------------------------------ MMA issuers (warps 5, 6)
 // K-steps [k0, k0 + kQkChunk) of the 36 (16 dims each) of QK for the page in stage s into
 // score buffer sb; the last chunk commits the buffer's QkDone.
 template <class C, int k0>
 __device__ __forceinline__ void issue_qk_chunk(const Smem<C>& sh, uint32_t tmem, uint32_t s, uint32_t sb) {
-    constexpr int kN = C::kN;
     constexpr uint32_t kIdesc = ptx::idesc_bf16(128, 64, false, false);
     ptx::tc_fence_after();
     const uint32_t d = tmem + C::kColS + 64 * sb;
@@ -320,9 +324,19 @@ __device__ __forceinline__ void issue_pv(const Smem<C>& sh, uint32_t tmem, uint3
     ptx::mma_commit(sh.bar(kBarPvDone));
 }
 
+// Bounded wait of an issuer thread: also gives up when another role has.
 template <class C>
-__device__ __forceinline__ void run_mma(const DecodeParams& p, const Smem<C>& sh, uint32_t tmem) {
-    constexpr int kN = C::kN;
+__device__ __forceinline__ bool issuer_wait(const Smem<C>& sh, uint32_t bar, uint32_t parity,
+                                            uint32_t where) {
+    return wait_bar(sh, bar, parity, where);
+}
+
+// QK issuer (warp 5, one thread): each page's QK as soon as its stage landed (and, for an
+// FP8 cache, was widened) and its score buffer was read out. PVs come from their own
+// thread (run_pv), so a P that is ready while a QK is being issued does not wait for the
+// whole QK to be issued first.
+template <class C>
+__device__ __forceinline__ void run_qk(const DecodeParams& p, const Smem<C>& sh, uint32_t tmem) {
     ItemIter iter(p, (int)blockIdx.x, (int)gridDim.x);
     Item it;
     uint32_t g = 0, gs = 0, items = 0;
@@ -330,61 +344,23 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Smem<C>& sh
     bool ok = true;
     while (ok && iter.next(it)) {
         // the item's q rows were moved out of their slot: free it
-        if (!wait_bar(sh, sh.bar(kBarQReady), items & 1u, 0x48u)) break;
+        if (!issuer_wait(sh, sh.bar(kBarQReady), items & 1u, 0x48u)) break;
         ptx::tc_fence_after();
         ptx::mbar_arrive(sh.bar(kBarFree + g % C::kStages));
         ++g;
         const uint32_t n = (uint32_t)it.pages();
-        uint32_t qk = 0, kc = 0, pv = 0;   // QKs and PVs issued (kc: chunks of a started QK)
-        bool o_free = items == 0;          // the previous item's O^T must be read out first
-        uint64_t t0 = 0;
-        uint32_t idle = 0;
-        while (pv < n) {
-            if (!o_free && ptx::mbar_test_wait(sh.bar(kBarOFree), (items - 1) & 1u)) {
-                ptx::tc_fence_after();
-                o_free = true;
-            }
+        for (uint32_t qk = 0; qk < n && ok; ++qk) {
             const uint32_t gq = g + qk, Sq = gs + qk;
-            bool can_qk = false;
-            if (qk < n) {
-                if (kc > 0) {
-                    can_qk = true;                         // continue the QK in progress
-                } else {
-                    // its score buffer must be free: S of step Sq - kSBufs read out
-                    bool sfree;
-                    if constexpr (C::kSBufs == 2) sfree = qk < pv + 2;
-                    else sfree = Sq == 0 || ptx::mbar_test_wait(sh.bar(kBarSFree), (Sq - 1) & 1u);
-                    const uint32_t st = gq % C::kStages;
-                    can_qk = sfree && ptx::mbar_test_wait(sh.bar(kBarFull + st), (gq / C::kStages) & 1u);
-                    if constexpr (C::kF8)
-                        can_qk = can_qk && ptx::mbar_test_wait(sh.bar(kBarDqFull + st), (dq_par >> st) & 1u);
-                }
+            const uint32_t st = gq % C::kStages, sb = Sq % C::kSBufs;
+            // its score buffer must be free: S of step Sq - kSBufs read out
+            if (Sq >= (uint32_t)C::kSBufs &&
+                !issuer_wait(sh, sh.bar(kBarSFree + sb), ((Sq / C::kSBufs) - 1u) & 1u, 0x49u)) { ok = false; break; }
+            if (!issuer_wait(sh, sh.bar(kBarFull + st), (gq / C::kStages) & 1u, 0x4bu)) { ok = false; break; }
+            if constexpr (C::kF8) {
+                if (!issuer_wait(sh, sh.bar(kBarDqFull + st), (dq_par >> st) & 1u, 0x4cu)) { ok = false; break; }
+                dq_par ^= 1u << st;
             }
-            if (pv < qk && (pv > 0 || o_free) &&
-                ptx::mbar_test_wait(sh.bar(kBarPReady), (gs + pv) & 1u)) {
-                issue_pv(sh, tmem, (g + pv) % C::kStages, pv == 0);
-                ++pv;
-                idle = 0;
-            } else if (can_qk) {
-                // a whole QK at once: slipping PVs in between its chunks was measured to
-                // slow the tensor pipe far more than it freed stages early
-                for (uint32_t ck = kc; ck < 4; ++ck)
-                    issue_qk_chunk(sh, tmem, gq % C::kStages, Sq % C::kSBufs, ck);
-                if constexpr (C::kF8) dq_par ^= 1u << (gq % C::kStages);
-                kc = 0;
-                ++qk;
-                idle = 0;
-            } else if ((++idle & 1023u) == 0) {
-                if (*sh.abort_flag()) { ok = false; break; }
-                const uint64_t now = ptx::globaltimer();
-                if (idle == 1024u) t0 = now;
-                else if (now - t0 > sh.wait_limit) {
-                    *sh.abort_flag() = 1;
-                    record_error(kErrTimeout, 0x49u);
-                    ok = false;
-                    break;
-                }
-            }
+            for (uint32_t ck = 0; ck < 4; ++ck) issue_qk_chunk(sh, tmem, st, sb, ck);
         }
         g += n;
         gs += n;
@@ -393,6 +369,32 @@ __device__ __forceinline__ void run_mma(const DecodeParams& p, const Smem<C>& sh
     // every MMA this thread issued is complete before the CTA may finish
     ptx::mma_commit(sh.bar(kBarDrain));
     drain_wait(sh, sh.bar(kBarDrain), 0, 0x4au);
+}
+
+// PV issuer (warp 6, one thread): each page's PV as soon as its P is written (and, for an
+// item's first page, the previous item's O^T was read out).
+template <class C>
+__device__ __forceinline__ void run_pv(const DecodeParams& p, const Smem<C>& sh, uint32_t tmem) {
+    ItemIter iter(p, (int)blockIdx.x, (int)gridDim.x);
+    Item it;
+    uint32_t g = 0, gs = 0, items = 0;
+    bool ok = true;
+    while (ok && iter.next(it)) {
+        ++g;                                   // the item's q slot
+        const uint32_t n = (uint32_t)it.pages();
+        for (uint32_t pv = 0; pv < n; ++pv) {
+            if (pv == 0 && items > 0 &&
+                !issuer_wait(sh, sh.bar(kBarOFree), (items - 1) & 1u, 0x4du)) { ok = false; break; }
+            if (!issuer_wait(sh, sh.bar(kBarPReady), (gs + pv) & 1u, 0x4eu)) { ok = false; break; }
+            ptx::tc_fence_after();
+            issue_pv(sh, tmem, (g + pv) % C::kStages, pv == 0);
+        }
+        g += n;
+        gs += n;
+        ++items;
+    }
+    ptx::mma_commit(sh.bar(kBarDrain + 1));
+    drain_wait(sh, sh.bar(kBarDrain + 1), 0, 0x4fu);
 }
 
 // ------------------------------------------------------------------ row group (warps 0-3)
@@ -434,7 +436,6 @@ __device__ __forceinline__ float pick(const float (&a)[K], int i) {
 // both sides are 1 KB aligned and row l keeps its row % 8, so the swizzle carries over).
 template <class C>
 __device__ __forceinline__ void move_q(const Smem<C>& sh, const RowCtx<C>& c, uint32_t s) {
-    constexpr int kN = C::kN;
     const uint32_t st = sh.stage(s);
     const int src_row = c.row;                     // < 32 kRowWarps; >= kN reads padding
 #pragma unroll 1
@@ -571,10 +572,8 @@ __device__ __forceinline__ bool row_step(const DecodeParams& p, const Smem<C>& s
     ptx::tc_fence_after();
     uint32_t sv[kTok];
     tmem_ld_cols<kTok>(c.tmem + c.lane_base + C::kColS + 64 * sb + c.copy * kTok, sv);
-    if constexpr (C::kSBufs == 1) {
-        ptx::tc_fence_before();                    // S read out before QK of S+1 rewrites it
-        warp_arrive(sh.bar(kBarSFree));
-    }
+    ptx::tc_fence_before();                        // S read out before a later QK rewrites it
+    warp_arrive(sh.bar(kBarSFree + sb));
     const int page = it.k_lo + (int)j;
     const int lim = n_vis - page * kBlock - c.copy * kTok;    // valid tokens of the slice [0, lim)
     const float m_own = pick(tr.m, c.own);
@@ -771,7 +770,6 @@ __device__ __forceinline__ bool epilogue(const DecodeParams& p, const Smem<C>& s
 
 template <class C>
 __device__ __forceinline__ void run_rows(const DecodeParams& p, const Smem<C>& sh, uint32_t tmem) {
-    constexpr int kN = C::kN;
     RowCtx<C> c;
     c.tmem = tmem;
     c.tid = (int)threadIdx.x;
@@ -847,7 +845,6 @@ __global__ void __launch_bounds__(C::kBlockThreads, 1)
 decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
               const __grid_constant__ CUtensorMap tm_scales, const __grid_constant__ CUtensorMap tm_rope,
               const __grid_constant__ CUtensorMap tm_q) {
-    constexpr int kN = C::kN;
     extern __shared__ uint8_t smem_raw[];
     Smem<C> sh;
     {
@@ -867,12 +864,14 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
         ptx::mbar_init(sh.bar(kBarQkDone + 1), 1);
         ptx::mbar_init(sh.bar(kBarPvDone), 1);
         ptx::mbar_init(sh.bar(kBarPReady), 4);
-        ptx::mbar_init(sh.bar(kBarSFree), 4);
+        ptx::mbar_init(sh.bar(kBarSFree + 0), 4);
+        ptx::mbar_init(sh.bar(kBarSFree + 1), 4);
         ptx::mbar_init(sh.bar(kBarQReady), 4);
         ptx::mbar_init(sh.bar(kBarOFree), 4);
         ptx::mbar_init(sh.bar(kBarDecide), 4);
         ptx::mbar_init(sh.bar(kBarEpi), 4);
-        ptx::mbar_init(sh.bar(kBarDrain), 1);
+        ptx::mbar_init(sh.bar(kBarDrain + 0), 1);
+        ptx::mbar_init(sh.bar(kBarDrain + 1), 1);
         ptx::mbar_init(sh.bar(kBarStall), 1);
         ptx::mbar_init(sh.bar(kBarWiden), kWidenWarps);
         for (int i = 0; i < kMaxStages; ++i) ptx::mbar_init(sh.bar(kBarDqFull + i), kWidenWarps);
@@ -899,7 +898,9 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
     } else if (warp == kWarpProducer) {
         if (lane == 0) run_producer<C>(p, sh, &tm_page, &tm_scales, &tm_rope, &tm_q);
     } else if (warp == kWarpMma) {
-        if (lane == 0) run_mma<C>(p, sh, tmem);
+        if (lane == 0) run_qk<C>(p, sh, tmem);
+    } else if (warp == kWarpPv) {
+        if (lane == 0) run_pv<C>(p, sh, tmem);
     } else if (C::kF8 && warp >= kWarpWiden) {
         run_widen<C>(p, sh, (int)threadIdx.x - 32 * kWarpWiden);
     }

@@ -54,7 +54,6 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
                 int num_units, int in_smem,
                 int32_t* __restrict__ metadata, int32_t* __restrict__ num_splits) {
     __shared__ int64_t warp_sums[33];
-    __shared__ int64_t s_total;
     extern __shared__ int32_t dyn[];
     const int V = batch * tiles;
     const int overhead = overhead_pages(h_q, s_q);
@@ -90,7 +89,6 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
     if (threadIdx.x == 0) {
         if (carry > 0x7fffffffLL) { record_error(kErrBadInput, 0xfffffeu); carry = 0x7fffffff; }
         Cs[V] = (int32_t)carry;
-        s_total = carry;
     }
     __syncthreads();
     auto C = [&](int v) { return (int64_t)Cs[v]; };

@@ -184,7 +184,7 @@ int device_solo_ctas(int dev) {
     if (prepare_solo_kernel<solo::Cfg<64>>(dev)) {
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, solo::decode_kernel<solo::Cfg<64>>,
-                                                          solo::kThreads,
+                                                          solo::Cfg<64>::kBlockThreads,
                                                           solo::Cfg<64>::kSmemAlloc) == cudaSuccess &&
             per_sm >= 1 && per_sm * sms < ctas)
             ctas = per_sm * sms;
@@ -342,7 +342,7 @@ mla_status launch_solo(const DecodeParams& p, const void* q, const void* kcache,
     if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
         !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
         return MLA_ERR_CUDA;
-    solo::decode_kernel<C><<<ctas, solo::kThreads, C::kSmemAlloc, s>>>(p, tm_page, tm_page, tm_page, tm_q);
+    solo::decode_kernel<C><<<ctas, C::kBlockThreads, C::kSmemAlloc, s>>>(p, tm_page, tm_page, tm_page, tm_q);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
