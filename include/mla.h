@@ -119,7 +119,7 @@ int mla_num_work_units(int num_sms, int h_q, int s_q);
  *               [0..7]   header {num_units, tiles, batch, h_q, s_q, unit_cost,
  *                        item_overhead, tile_aligned}: a work sequence costs its pages
  *                        plus item_overhead (3 for the 2-CTA kernel; for the 1-CTA
- *                        kernel 1 up to 32 query rows, 3 for 33-64). With tiles > 1
+ *                        kernel 1 up to 32 query rows, 2 for 33-64). With tiles > 1
  *                        row tiles per sequence and at least `tiles` units
  *                        (tile_aligned = 1), tile t owns units
  *                        [floor(t U/tiles), floor((t+1) U/tiles)) and balances the

@@ -40,10 +40,11 @@ constexpr int kTileRows = 128;
 // kSoloMaxRows query rows), whose q rows ride in a slot of the page ring and whose
 // epilogue overlaps the next item's first QK, about 0.6 of a page with 16 rows (three
 // stages) but 2.5 pages with 64 rows (two stages, a 72 KB q slot and a 48 KB copy of the
-// q rows into shared memory).
+// q rows into shared memory). For 33-64 rows, 2 measured best once QK and PV got issuers
+// of their own (2, 3 and 4 timed).
 constexpr int kOverheadPages = 3;
 constexpr int kOverheadPagesSolo = 1;
-constexpr int kOverheadPagesSoloWide = 3;   // 1-CTA kernel, 33-64 query rows
+constexpr int kOverheadPagesSoloWide = 2;   // 1-CTA kernel, 33-64 query rows
 constexpr int kSoloMaxRows = 64;
 
 MLA_HD int overhead_pages(int h_q, int s_q) {

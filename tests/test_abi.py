@@ -153,9 +153,10 @@ def test_schedule_random_and_balanced():
         seen, nblk = _walk(meta, ns, lens, h_q, s_q)
         W = int(meta[5])
         # fixed cost per work sequence, in pages: 1 for the 1-CTA kernel up to 32 query
-        # rows per sequence, 3 for it with 33-64 rows and for the 2-CTA kernel; the header
+        # rows per sequence, 2 for it with 33-64 rows, 3 for the 2-CTA kernel; the header
         # records it
-        overhead = 1 if h_q * s_q <= 32 else 3
+        rows = h_q * s_q
+        overhead = 1 if rows <= 32 else 2 if rows <= 64 else 3
         assert int(meta[6]) == overhead
         total = sum(overhead + n for n in nblk)
         T = int(meta[1])
