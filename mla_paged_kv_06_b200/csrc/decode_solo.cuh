@@ -510,12 +510,11 @@ __device__ __forceinline__ void widen_units(uint32_t tile_row, int row, int part
 
 // FP8 cache: widens the page in the stage of ring slot g in place, into the 9-tile
 // swizzled bf16 layout QK and PV read (the rope tile arrived by TMA). The widening warps
-// give each row kWidenWarps / 2 threads, each a contiguous share of each tile's 64 dims. Widened tiles 4-7 overwrite
-// codes, so the tiles go in order and the row group syncs where an output meets codes
-// not yet read: after the scales are read (tile 3 covers them), after tiles 0-3 (tiles 4
-// and 5 cover codes 0-3), after tiles 4-5 (tile 6 covers codes 4-5), and before tile 7
-// (it covers codes 6-7; its own codes wait in registers). Rows past the sequence end are
-// written as zeros (their codes may be anything, NaN included).
+// give each row kWidenWarps / 2 threads, each a contiguous share of each tile's 64 dims.
+// Every thread first reads its scales and all its codes into registers; tiles 0-2 lie
+// below every input and are written at once; tiles 3-7 cover the scales and the codes,
+// so they follow one sync of the widening warps (all inputs read). Rows past the
+// sequence end are written as zeros (their codes may be anything, NaN included).
 template <class C>
 __device__ __forceinline__ bool widen(const Smem<C>& sh, int tid, const Item& it, int page,
                                       uint32_t g, uint32_t& n_syncs) {
@@ -531,29 +530,21 @@ __device__ __forceinline__ bool widen(const Smem<C>& sh, int tid, const Item& it
     const uint4 scv = ptx::ld_shared_v4(st + kF8ScaleOff + (uint32_t)row * 16);
     const float sc[4] = {__uint_as_float(scv.x), __uint_as_float(scv.y), __uint_as_float(scv.z),
                          __uint_as_float(scv.w)};
-    auto codes = [&](int ch, uint4 (&w)[kU]) {
+    uint4 w[8][kU];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
         const uint32_t a = st + kF8CodeOff + (uint32_t)ch * 4096 + (uint32_t)row * 64 + (uint32_t)part * 16 * kU;
 #pragma unroll
-        for (int u = 0; u < kU; ++u) w[u] = ptx::ld_shared_v4(a + 16 * u);
-    };
-    auto tile = [&](int ch, const uint4 (&w)[kU]) {
-        widen_units<kU>(st + (uint32_t)ch * kBoxBytes + (uint32_t)row * 128, row, part, sc[ch >> 1], w, live);
-    };
-    if (!widen_sync(sh, n_syncs)) return false;
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch) { uint4 w[kU]; codes(ch, w); tile(ch, w); }
-    if (!widen_sync(sh, n_syncs)) return false;
-#pragma unroll
-    for (int ch = 4; ch < 6; ++ch) { uint4 w[kU]; codes(ch, w); tile(ch, w); }
-    if (!widen_sync(sh, n_syncs)) return false;
-    {
-        uint4 w6[kU], w7[kU];
-        codes(6, w6);
-        tile(6, w6);
-        codes(7, w7);
-        if (!widen_sync(sh, n_syncs)) return false;
-        tile(7, w7);
+        for (int u = 0; u < kU; ++u) w[ch][u] = ptx::ld_shared_v4(a + 16 * u);
     }
+    auto tile = [&](int ch) {
+        widen_units<kU>(st + (uint32_t)ch * kBoxBytes + (uint32_t)row * 128, row, part, sc[ch >> 1], w[ch], live);
+    };
+#pragma unroll
+    for (int ch = 0; ch < 3; ++ch) tile(ch);
+    if (!widen_sync(sh, n_syncs)) return false;
+#pragma unroll
+    for (int ch = 3; ch < 8; ++ch) tile(ch);
     ptx::fence_proxy_async_smem();           // the widened tiles visible to the MMA
     warp_arrive(sh.bar(kBarDqFull + s));
     return true;
