@@ -188,13 +188,16 @@ FULL = ["uniform", "v3", "spec", "skewed"]
 
 
 @pytest.mark.parametrize("h_q,s_q,num_sms,chunks", [
+    (16, 1, 2, 2), (16, 1, 3, 3), (16, 1, 4, 4), (16, 1, 5, 5), (32, 1, 4, 4),
+    (64, 1, 2, 2), (64, 1, 3, 3),
     (16, 1, 8, 8), (16, 1, 9, 9), (16, 1, 17, 17), (16, 1, 33, 33), (16, 1, 148, 129),
     (128, 2, 40, 10), (128, 2, 140, 34),
 ])
 def test_rows_merged_from_many_chunks(h_q, s_q, num_sms, chunks):
-    # One long sequence spread over every unit: the combine cuts a row of more than 8
-    # chunks into slices merged by separate CTAs and then merges the slices. Short
-    # sequences beside it keep the one-pass merge.
+    # One long sequence spread over 2 to 148 units, merged by the combine: a row of more
+    # than 8 chunks is cut into slices merged by separate CTAs, then the slices are
+    # merged (the second run on the same schedule checks that the slice counters start
+    # from zero again). Short sequences beside it keep the one-pass merge.
     mla = _mla()
     lens = [40960, 100, 0, 64]
     x = wl.make_paged_inputs(lens, s_q, h_q, seed=chunks + h_q, causal=s_q > 1,
@@ -203,9 +206,17 @@ def test_rows_merged_from_many_chunks(h_q, s_q, num_sms, chunks):
     _, ns = mla.mla_plan_host(lens, h_q, s_q, mla.mla_num_work_units(nsm, h_q, s_q))
     if nsm == num_sms:
         assert int(ns[1] - ns[0]) == chunks      # the first sequence's chunks (tile 0)
-    out, lse = run(x, num_sms=nsm)
+    d = to_dev(x)
+    meta, ns = mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm)
+    res = []
+    for _ in range(2):                           # one schedule, two calls
+        res.append(mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"],
+                                      x.scale, x.causal, meta, ns, num_sms=nsm))
+        torch.cuda.synchronize()
+        st, word = mla.mla_get_last_device_error()
+        assert st == 0, f"device error {mla.status_string(st)} word={word:#x}"
+    (out, lse), (out2, lse2) = res
     compare(out, lse, *oracle_all(x), what=f"{h_q}/{s_q}/{nsm}")
-    out2, lse2 = run(x, num_sms=nsm)
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
 
 
