@@ -65,7 +65,6 @@ constexpr uint32_t kStageBytes = 9 * kBoxBytes;      // one page: 64 tokens x 57
 constexpr uint32_t kSmemLimit = 232448;              // sm_100 per-block opt-in maximum
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxStages = 3;
-constexpr int kQkChunk = 9;                          // K-steps of QK per issue burst
 // An FP8 page lands in its own stage and is widened there: its codes as 8 tiles of 64 rows
 // x 64 bytes at [32, 64) KB (tile c = latent dims [64 c, 64 c + 64)), its scales as 64 rows
 // x 16 bytes at [31, 32) KB, its rope dims (bf16) already in the rope tile at [64, 72) KB.
@@ -125,7 +124,8 @@ enum : uint32_t {
     kBarStall = kBarDrain + 2,           // never completes (the timeout test hook waits on it)
     kBarWiden = kBarStall + 1,           // FP8 cache: the widening warps' syncs inside a page
     kBarDqFull = kBarWiden + 1,          // [kMaxStages] FP8 cache: a stage's page widened (kWidenWarps arrivals)
-    kNumBars = kBarDqFull + kMaxStages
+    kBarDqHalf = kBarDqFull + kMaxStages,  // [kMaxStages] FP8 cache: its tiles 0-2 widened
+    kNumBars = kBarDqHalf + kMaxStages
 };
 // misc area: barriers [0, 256), tmem base at 256, abort flag at 260; partial maxima
 // [2 parity][4 copies][64 rows] f32 at 512; partial row sums [2 sums][4 copies][64] at
@@ -266,16 +266,16 @@ __device__ __forceinline__ void run_producer(const DecodeParams& p, const Smem<C
 }
 
 // ------------------------------------------------------------------ MMA issuers (warps 5, 6)
-// K-steps [k0, k0 + kQkChunk) of the 36 (16 dims each) of QK for the page in stage s into
-// score buffer sb; the last chunk commits the buffer's QkDone.
-template <class C, int k0>
-__device__ __forceinline__ void issue_qk_chunk(const Smem<C>& sh, uint32_t tmem, uint32_t s, uint32_t sb) {
+// K-steps [k0, k1) of the 36 (16 dims each) of QK for the page in stage s into score
+// buffer sb; the part that ends at 36 commits the buffer's QkDone.
+template <class C, int k0, int k1>
+__device__ __forceinline__ void issue_qk_range(const Smem<C>& sh, uint32_t tmem, uint32_t s, uint32_t sb) {
     constexpr uint32_t kIdesc = ptx::idesc_bf16(128, 64, false, false);
     ptx::tc_fence_after();
     const uint32_t d = tmem + C::kColS + 64 * sb;
     const uint32_t st = sh.stage(s);
 #pragma unroll
-    for (int k = k0; k < k0 + kQkChunk; ++k) {
+    for (int k = k0; k < k1; ++k) {
         const uint64_t bdesc = ptx::smem_desc(st + (k >> 2) * kBoxBytes + (k & 3) * 32, 16, 1024, 2);
         if (k < 4 * C::kQtChunks) {
             ptx::mma_ts(d, tmem + C::kColQ + 8 * k, bdesc, kIdesc, k > 0 ? 1u : 0u);
@@ -286,19 +286,7 @@ __device__ __forceinline__ void issue_qk_chunk(const Smem<C>& sh, uint32_t tmem,
             ptx::mma_ss(d, adesc, bdesc, kIdesc, k > 0 ? 1u : 0u);
         }
     }
-    if constexpr (k0 + kQkChunk == 36) ptx::mma_commit(sh.bar(kBarQkDone + sb));
-}
-
-template <class C>
-__device__ __forceinline__ void issue_qk_chunk(const Smem<C>& sh, uint32_t tmem, uint32_t s,
-                                               uint32_t sb, uint32_t chunk) {
-    static_assert(4 * kQkChunk == 36, "four chunks per QK");
-    switch (chunk) {
-        case 0: issue_qk_chunk<C, 0>(sh, tmem, s, sb); break;
-        case 1: issue_qk_chunk<C, kQkChunk>(sh, tmem, s, sb); break;
-        case 2: issue_qk_chunk<C, 2 * kQkChunk>(sh, tmem, s, sb); break;
-        default: issue_qk_chunk<C, 3 * kQkChunk>(sh, tmem, s, sb); break;
-    }
+    if constexpr (k1 == 36) ptx::mma_commit(sh.bar(kBarQkDone + sb));
 }
 
 // O^T += V^T P^T for the page in stage s; `first` starts the item's accumulation.
@@ -357,10 +345,16 @@ __device__ __forceinline__ void run_qk(const DecodeParams& p, const Smem<C>& sh,
                 !issuer_wait(sh, sh.bar(kBarSFree + sb), ((Sq / C::kSBufs) - 1u) & 1u, 0x49u)) { ok = false; break; }
             if (!issuer_wait(sh, sh.bar(kBarFull + st), (gq / C::kStages) & 1u, 0x4bu)) { ok = false; break; }
             if constexpr (C::kF8) {
-                if (!issuer_wait(sh, sh.bar(kBarDqFull + st), (dq_par >> st) & 1u, 0x4cu)) { ok = false; break; }
+                // the K-steps of the first three tiles as soon as those are widened
+                const uint32_t par = (dq_par >> st) & 1u;
                 dq_par ^= 1u << st;
+                if (!issuer_wait(sh, sh.bar(kBarDqHalf + st), par, 0x4du)) { ok = false; break; }
+                issue_qk_range<C, 0, 12>(sh, tmem, st, sb);
+                if (!issuer_wait(sh, sh.bar(kBarDqFull + st), par, 0x4cu)) { ok = false; break; }
+                issue_qk_range<C, 12, 36>(sh, tmem, st, sb);
+            } else {
+                issue_qk_range<C, 0, 36>(sh, tmem, st, sb);
             }
-            for (uint32_t ck = 0; ck < 4; ++ck) issue_qk_chunk(sh, tmem, st, sb, ck);
         }
         g += n;
         gs += n;
@@ -542,6 +536,8 @@ __device__ __forceinline__ bool widen(const Smem<C>& sh, int tid, const Item& it
     };
 #pragma unroll
     for (int ch = 0; ch < 3; ++ch) tile(ch);
+    ptx::fence_proxy_async_smem();           // tiles 0-2 visible to the MMA: QK may start
+    warp_arrive(sh.bar(kBarDqHalf + s));
     if (!widen_sync(sh, n_syncs)) return false;
 #pragma unroll
     for (int ch = 3; ch < 8; ++ch) tile(ch);
@@ -865,7 +861,10 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
         ptx::mbar_init(sh.bar(kBarDrain + 1), 1);
         ptx::mbar_init(sh.bar(kBarStall), 1);
         ptx::mbar_init(sh.bar(kBarWiden), kWidenWarps);
-        for (int i = 0; i < kMaxStages; ++i) ptx::mbar_init(sh.bar(kBarDqFull + i), kWidenWarps);
+        for (int i = 0; i < kMaxStages; ++i) {
+            ptx::mbar_init(sh.bar(kBarDqFull + i), kWidenWarps);
+            ptx::mbar_init(sh.bar(kBarDqHalf + i), kWidenWarps);
+        }
         *sh.abort_flag() = 0;
         ptx::fence_mbarrier_init_cluster();
         ptx::prefetch_tensormap(&tm_page);
