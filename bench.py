@@ -9,7 +9,10 @@ query heads, one shared 576-dim latent head, lengths uniform in [1, 8192], 64-to
 bf16 pages randomly permuted in the pool. Inputs are seeded synthetic data.
 
 Rank 0 prints one JSON line. `value` is algorithmic HBM bytes (every visible KV row
-once, q, out, lse) of all ranks' steps divided by the max-over-ranks device time;
+once, q, out, lse) of all ranks' steps divided by the max-over-ranks device time. A step
+that reads at least twice the 126 MB L2 runs back to back with the others (inputs larger
+than L2); smaller ones get an untimed 256 MB L2 write before each, and every workload is
+also reported with that flush (`l2_write_flush`);
 `roofline` relates the decode call to the measured peaks; `e2e` repeats the measurement
 with q, block table and lengths copied from pinned host memory and the outputs read
 back every step; `cpu_baseline` times the fp64 CPU oracle on a bounded sample.
@@ -35,6 +38,8 @@ from mla_paged_kv_06_b200 import workloads as wl  # noqa: E402
 from mla_paged_kv_06_b200.shard import max_over_ranks, rank_seed  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
+L2_BYTES = 126 << 20                # B200 L2
+HEADSTART_CYCLES_PER_STEP = 200_000 # an untimed sleep kernel of ~100 us per queued step
 kBlockRoom = 64                     # tokens per page
 LAUNCHES_PER_STEP = 3               # metadata, split kernel, combine kernel
 SPLIT_KV_WORLD = 4                  # ranks of the split-KV-across-devices measurement
@@ -305,6 +310,41 @@ NOMINAL_HBM_GBS = 8000.0
 NOMINAL_BF16_TFLOPS = 2250.0
 
 
+def flush_free(nbytes):
+    """True when a step reads at least twice L2: then steps run back to back with no flush
+    (their inputs exceed L2), otherwise an untimed write of 256 MB flushes L2 before each."""
+    return nbytes >= 2 * L2_BYTES
+
+
+def l2_note(nbytes, no_flush):
+    if no_flush:
+        return (f"no flush: each step reads {nbytes / 1e6:.0f} MB, "
+                f"{nbytes / L2_BYTES:.1f}x the 126 MB L2; the steps run back to back, queued "
+                "behind an untimed sleep kernel so that no host gap enters the timing")
+    return ("L2 flushed (256 MB write, untimed) before every step")
+
+
+def time_steps(parts, steps, flush, stream, no_flush):
+    """Times `steps` steps; a step runs the callables in `parts` in order on `stream`, with
+    a CUDA event before the first and after each. Returns, per part, the list of its
+    per-step times in ms. With no_flush the steps run back to back (a sleep kernel queued
+    first lets the host enqueue them all before the first starts); otherwise an untimed
+    256 MB write flushes L2 before each step."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+          for _ in range(steps)]
+    if no_flush:
+        torch.cuda._sleep(HEADSTART_CYCLES_PER_STEP * steps)
+    for e in ev:
+        if not no_flush:
+            flush.zero_()
+        e[0].record(stream)
+        for i, f in enumerate(parts):
+            f()
+            e[i + 1].record(stream)
+    torch.cuda.synchronize()
+    return [[e[i].elapsed_time(e[i + 1]) for e in ev] for i in range(len(parts))]
+
+
 def roofline_fracs(nbytes, nflops, seconds, hbm_peak, tf_peak):
     t_bytes = nbytes / (hbm_peak * 1e9)
     t_flops = nflops / (tf_peak * 1e12)
@@ -316,11 +356,21 @@ def roofline_fracs(nbytes, nflops, seconds, hbm_peak, tf_peak):
             "roofline_frac_nominal": max(n_bytes, n_flops) / seconds}
 
 
+def flushed_entry(nbytes, meta_ms, decode_ms, hbm_peak):
+    """The same workload timed with a 256 MB L2 write before every step. Evicting those
+    dirty lines writes up to 126 MB back to HBM inside the timed decode call."""
+    t = statistics.mean(decode_ms) / 1e3
+    return {"us_per_call": statistics.median([a + b for a, b in zip(meta_ms, decode_ms)]) * 1e3,
+            "us_per_call_decode": statistics.median(decode_ms) * 1e3,
+            "GB/s": nbytes / t / 1e9, "hbm_frac": nbytes / t / 1e9 / hbm_peak}
+
+
 def time_config(mla, name, seed, flush, stream, steps, warmup, hbm_peak, tf_peak,
                 cpu_seconds, with_cpu):
-    """One workload's decode timed the way the main measurement times it (L2 flushed,
-    untimed, before each step; metadata and decode call timed with CUDA events on the
-    launching stream), reported against its own roofline."""
+    """One workload's decode timed the way the main measurement times it (metadata and
+    decode call timed with CUDA events on the launching stream; no flush when the step
+    reads at least twice L2, else an untimed L2 flush before each step; the flushed
+    timing is also reported), against its own roofline."""
     x = wl.make_workload(name, seed=seed)
     d = dict(q=x.q.cuda(), kcache=x.kcache.cuda(), block_table=x.block_table.cuda(),
              seqlens=x.seqlens.cuda())
@@ -332,40 +382,32 @@ def time_config(mla, name, seed, flush, stream, steps, warmup, hbm_peak, tf_peak
                      device="cuda")
     out = torch.empty((x.batch, x.s_q, x.h_q, 512), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
-    for _ in range(max(warmup, 3)):
-        flush.zero_()
-        mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
-        mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
-                           x.causal, meta, ns, ws, out, lse)
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for k in range(steps):
-        flush.zero_()
-        e0, e1, e2 = ev[k]
-        e0.record(stream)
-        mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
-        e1.record(stream)
-        mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
-                           x.causal, meta, ns, ws, out, lse)
-        e2.record(stream)
-    torch.cuda.synchronize()
+    nbytes, nflops = wl.algorithmic_work(x.seqlens, x.s_q, x.h_q, x.causal)
+    no_flush = flush_free(nbytes)
+    parts = [lambda: mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns),
+             lambda: mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"],
+                                        x.scale, x.causal, meta, ns, ws, out, lse)]
+    time_steps(parts, max(warmup, 3), flush, stream, no_flush)
+    meta_ms, decode_ms = time_steps(parts, steps, flush, stream, no_flush)
+    fl_meta_ms, fl_decode_ms = (time_steps(parts, steps, flush, stream, False) if no_flush
+                                else (meta_ms, decode_ms))
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error in {name}: {mla.status_string(st)} {word:#x}")
-    step_ms = [a.elapsed_time(c) for a, _, c in ev]
-    decode_ms = [b.elapsed_time(c) for _, b, c in ev]
-    nbytes, nflops = wl.algorithmic_work(x.seqlens, x.s_q, x.h_q, x.causal)
+    step_ms = [a + b for a, b in zip(meta_ms, decode_ms)]
     t = statistics.mean(decode_ms) / 1e3
     rows = x.s_q * x.h_q
     entry = {"workload": workload_config(x, name)["workload"], "batch": x.batch,
              "s_q": x.s_q, "h_q": x.h_q, "total_tokens": int(x.seqlens.sum()),
              "kernel": "1-CTA (rows <= 64)" if rows <= 64 else "2-CTA pairs",
+             "l2": l2_note(nbytes, no_flush),
              "us_per_call": statistics.median(step_ms) * 1e3,
              "us_per_call_decode": statistics.median(decode_ms) * 1e3,
+             "us_per_call_metadata": statistics.median(meta_ms) * 1e3,
              "GB/s": nbytes / t / 1e9, "TFLOPS": nflops / t / 1e12,
              "algorithmic_bytes": nbytes, "algorithmic_flops": nflops,
-             "roofline": roofline_fracs(nbytes, nflops, t, hbm_peak, tf_peak)}
+             "roofline": roofline_fracs(nbytes, nflops, t, hbm_peak, tf_peak),
+             "l2_write_flush": flushed_entry(nbytes, fl_meta_ms, fl_decode_ms, hbm_peak)}
     if with_cpu:
         entry["cpu_baseline"] = cpu_baseline(x, cpu_seconds)
     del d, ws, out, lse
@@ -430,8 +472,10 @@ def time_fp8(mla, seed, flush, stream, steps, warmup, hbm_peak):
             "us_per_call": us, "GB/s": gbs, "hbm_frac": gbs / hbm_peak,
             "algorithmic_bytes": nbytes,
             "bf16_cache_bytes_same_workload": tokens * 1152 + rows_total * (1152 + 1024 + 4),
-            "note": "metadata + mla_decode_fwd_fp8 per call, L2 flushed before each; the "
-                    "cache was quantized on the GPU by mla_kv_append_fp8"}
+            "note": "mla_decode_fwd_fp8 per call, L2 flushed (256 MB write) before each: "
+                    "its reads are under twice L2 (compare the uniform entry's "
+                    "l2_write_flush figure); the cache was quantized on the GPU by "
+                    "mla_kv_append_fp8"}
 
 
 def main():
@@ -467,42 +511,28 @@ def main():
     stream = torch.cuda.current_stream()
     nbytes, nflops = wl.algorithmic_work(x.seqlens, x.s_q, x.h_q, x.causal)
 
-    def step():
-        mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
-        mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
-                           x.causal, meta, ns, ws, out, lse)
-
-    for _ in range(max(args.warmup, 3)):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
+    no_flush = flush_free(nbytes)
+    parts = [lambda: mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns),
+             lambda: mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"],
+                                        x.scale, x.causal, meta, ns, ws, out, lse)]
+    time_steps(parts, max(args.warmup, 3), flush, stream, no_flush)
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error during warm-up: {mla.status_string(st)} {word:#x}")
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for k in range(args.steps):
-            flush.zero_()                                  # untimed L2 flush
-            e0, e1, e2 = ev[k]
-            e0.record(stream)
-            mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
-            e1.record(stream)
-            mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
-                               x.causal, meta, ns, ws, out, lse)
-            e2.record(stream)
-        torch.cuda.synchronize()
+        meta_ms, decode_ms = time_steps(parts, args.steps, flush, stream, no_flush)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
-    decode_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
-    meta_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    step_ms = [a + b for a, b in zip(meta_ms, decode_ms)]
     total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
+    # the same steps with a 256 MB L2 write before each (every rank, in the same order)
+    fl_meta_ms, fl_decode_ms = (time_steps(parts, args.steps, flush, stream, False)
+                                if no_flush else (meta_ms, decode_ms))
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error during timing: {mla.status_string(st)} {word:#x}")
@@ -667,13 +697,13 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 q and cache; seeded lengths and page permutation)",
             "config": dict(workload_config(x, args.workload),
-                           l2="L2 flushed (256 MB write, untimed) before every step; the step's "
-                              "KV rows exceed L2", parallelism=f"replicas x{world}"),
+                           l2=l2_note(nbytes, no_flush), parallelism=f"replicas x{world}"),
             "tflops": nflops * args.steps * world / (total_ms / 1e3) / 1e12,
             "us_per_call": statistics.median(step_ms) * 1e3,
             "us_per_call_decode": statistics.median(decode_ms) * 1e3,
             "us_per_call_metadata": statistics.median(meta_ms) * 1e3,
             "roofline": roof,
+            "l2_write_flush": flushed_entry(nbytes, fl_meta_ms, fl_decode_ms, hbm_peak),
             "e2e": {"value": nbytes * args.steps * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / args.steps,
@@ -700,11 +730,14 @@ def main():
         main_entry = {"workload": line["config"]["workload"], "batch": x.batch, "s_q": x.s_q,
                       "h_q": x.h_q, "total_tokens": int(x.seqlens.sum()),
                       "kernel": "1-CTA (rows <= 64)" if x.s_q * x.h_q <= 64 else "2-CTA pairs",
+                      "l2": line["config"]["l2"],
                       "us_per_call": line["us_per_call"],
                       "us_per_call_decode": line["us_per_call_decode"],
+                      "us_per_call_metadata": line["us_per_call_metadata"],
                       "GB/s": achieved_gbs, "TFLOPS": achieved_tf,
                       "algorithmic_bytes": nbytes, "algorithmic_flops": nflops,
-                      "roofline": roofline_fracs(nbytes, nflops, avg_decode_s, hbm_peak, tf_peak)}
+                      "roofline": roofline_fracs(nbytes, nflops, avg_decode_s, hbm_peak, tf_peak),
+                      "l2_write_flush": line["l2_write_flush"]}
         if "cpu_baseline" in line:
             main_entry["cpu_baseline"] = line["cpu_baseline"]
         line["configs"] = {n: (main_entry if n == args.workload else configs[n])
