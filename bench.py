@@ -4,9 +4,10 @@
 
 One step = one pass of the whole hot path over one batch: the split-KV scheduler
 (mla_get_metadata), the split kernel and the LSE combine (mla_decode_fwd), all through
-the C ABI. The default workload is DeepSeek-V3-shaped decode: batch 128, s_q 1, 128
-query heads, one shared 576-dim latent head, lengths uniform in [1, 8192], 64-token
-bf16 pages randomly permuted in the pool. Inputs are seeded synthetic data.
+the C ABI, captured once as a CUDA graph and replayed per step. The default workload is
+DeepSeek-V3-shaped decode: batch 128, s_q 1, 128 query heads, one shared 576-dim latent
+head, lengths uniform in [1, 8192], 64-token bf16 pages randomly permuted in the pool.
+Inputs are seeded synthetic data.
 
 Rank 0 prints one JSON line. `value` is algorithmic HBM bytes (every visible KV row
 once, q, out, lse) of all ranks' steps divided by the max-over-ranks device time. A step
@@ -40,6 +41,10 @@ from mla_paged_kv_06_b200.shard import max_over_ranks, rank_seed  # noqa: E402
 L2_FLUSH_BYTES = 256 << 20          # > 126 MB L2
 L2_BYTES = 126 << 20                # B200 L2
 HEADSTART_CYCLES_PER_STEP = 200_000 # an untimed sleep kernel of ~100 us per queued step
+TIMING_NOTE = ("each step is one replay of a CUDA graph of the C-ABI calls mla_get_metadata "
+               "+ mla_decode_fwd (metadata, split and combine kernels), between CUDA events "
+               "on the launching stream; the decode call and the metadata call are also "
+               "timed alone the same way")
 kBlockRoom = 64                     # tokens per page
 LAUNCHES_PER_STEP = 3               # metadata, split kernel, combine kernel
 SPLIT_KV_WORLD = 4                  # ranks of the split-KV-across-devices measurement
@@ -324,25 +329,60 @@ def l2_note(nbytes, no_flush):
     return ("L2 flushed (256 MB write, untimed) before every step")
 
 
-def time_steps(parts, steps, flush, stream, no_flush):
-    """Times `steps` steps; a step runs the callables in `parts` in order on `stream`, with
-    a CUDA event before the first and after each. Returns, per part, the list of its
-    per-step times in ms. With no_flush the steps run back to back (a sleep kernel queued
-    first lets the host enqueue them all before the first starts); otherwise an untimed
-    256 MB write flushes L2 before each step."""
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+def capture(parts):
+    """A CUDA graph of the calls in `parts`, made in order (their launches through the C
+    ABI are recorded once and replayed as one unit, as a serving loop replays its step)."""
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in parts:
+            f()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_replays(g, steps, flush, stream, no_flush):
+    """Per-step times (ms) of `steps` replays of graph g, each between two CUDA events on
+    `stream`. With no_flush the replays run back to back (a sleep kernel queued first lets
+    the host enqueue them all before the first starts); otherwise an untimed 256 MB write
+    flushes L2 before each."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     if no_flush:
         torch.cuda._sleep(HEADSTART_CYCLES_PER_STEP * steps)
-    for e in ev:
+    for a, b in ev:
         if not no_flush:
             flush.zero_()
-        e[0].record(stream)
-        for i, f in enumerate(parts):
-            f()
-            e[i + 1].record(stream)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
     torch.cuda.synchronize()
-    return [[e[i].elapsed_time(e[i + 1]) for e in ev] for i in range(len(parts))]
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+class StepTimer:
+    """The step (metadata + decode call), the decode call alone and the metadata call
+    alone, each captured as a CUDA graph after `warmup` eager steps."""
+
+    def __init__(self, meta_fn, decode_fn, warmup, flush, stream, no_flush):
+        for _ in range(max(warmup, 3)):
+            if not no_flush:
+                flush.zero_()
+            meta_fn()
+            decode_fn()
+        torch.cuda.synchronize()
+        self.graphs = {"step": capture([meta_fn, decode_fn]), "decode": capture([decode_fn]),
+                       "metadata": capture([meta_fn])}
+        self.flush, self.stream, self.no_flush = flush, stream, no_flush
+        for g in self.graphs.values():
+            time_replays(g, 3, flush, stream, no_flush)
+
+    def time(self, which, steps, no_flush=None):
+        nf = self.no_flush if no_flush is None else no_flush
+        return time_replays(self.graphs[which], steps, self.flush, self.stream, nf)
+
+    def release(self):
+        self.graphs = {}
 
 
 def roofline_fracs(nbytes, nflops, seconds, hbm_peak, tf_peak):
@@ -356,11 +396,11 @@ def roofline_fracs(nbytes, nflops, seconds, hbm_peak, tf_peak):
             "roofline_frac_nominal": max(n_bytes, n_flops) / seconds}
 
 
-def flushed_entry(nbytes, meta_ms, decode_ms, hbm_peak):
+def flushed_entry(nbytes, step_ms, decode_ms, hbm_peak):
     """The same workload timed with a 256 MB L2 write before every step. Evicting those
     dirty lines writes up to 126 MB back to HBM inside the timed decode call."""
     t = statistics.mean(decode_ms) / 1e3
-    return {"us_per_call": statistics.median([a + b for a, b in zip(meta_ms, decode_ms)]) * 1e3,
+    return {"us_per_call": statistics.median(step_ms) * 1e3,
             "us_per_call_decode": statistics.median(decode_ms) * 1e3,
             "GB/s": nbytes / t / 1e9, "hbm_frac": nbytes / t / 1e9 / hbm_peak}
 
@@ -384,17 +424,18 @@ def time_config(mla, name, seed, flush, stream, steps, warmup, hbm_peak, tf_peak
     lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
     nbytes, nflops = wl.algorithmic_work(x.seqlens, x.s_q, x.h_q, x.causal)
     no_flush = flush_free(nbytes)
-    parts = [lambda: mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns),
-             lambda: mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"],
-                                        x.scale, x.causal, meta, ns, ws, out, lse)]
-    time_steps(parts, max(warmup, 3), flush, stream, no_flush)
-    meta_ms, decode_ms = time_steps(parts, steps, flush, stream, no_flush)
-    fl_meta_ms, fl_decode_ms = (time_steps(parts, steps, flush, stream, False) if no_flush
-                                else (meta_ms, decode_ms))
+    timer = StepTimer(
+        lambda: mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns),
+        lambda: mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"],
+                                   x.scale, x.causal, meta, ns, ws, out, lse),
+        warmup, flush, stream, no_flush)
+    step_ms, decode_ms, meta_ms = (timer.time(w, steps) for w in ("step", "decode", "metadata"))
+    fl = ({w: timer.time(w, steps, no_flush=False) for w in ("step", "decode")} if no_flush
+          else {"step": step_ms, "decode": decode_ms})
+    timer.release()
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error in {name}: {mla.status_string(st)} {word:#x}")
-    step_ms = [a + b for a, b in zip(meta_ms, decode_ms)]
     t = statistics.mean(decode_ms) / 1e3
     rows = x.s_q * x.h_q
     entry = {"workload": workload_config(x, name)["workload"], "batch": x.batch,
@@ -407,7 +448,7 @@ def time_config(mla, name, seed, flush, stream, steps, warmup, hbm_peak, tf_peak
              "GB/s": nbytes / t / 1e9, "TFLOPS": nflops / t / 1e12,
              "algorithmic_bytes": nbytes, "algorithmic_flops": nflops,
              "roofline": roofline_fracs(nbytes, nflops, t, hbm_peak, tf_peak),
-             "l2_write_flush": flushed_entry(nbytes, fl_meta_ms, fl_decode_ms, hbm_peak)}
+             "l2_write_flush": flushed_entry(nbytes, fl["step"], fl["decode"], hbm_peak)}
     if with_cpu:
         entry["cpu_baseline"] = cpu_baseline(x, cpu_seconds)
     del d, ws, out, lse
@@ -439,26 +480,15 @@ def time_fp8(mla, seed, flush, stream, steps, warmup, hbm_peak):
     out = torch.empty((x.batch, x.s_q, x.h_q, 512), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
 
-    # the schedule is computed once, as for the bf16 decode call's timing
-    mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
-
-    def call():
-        mla.mla_decode_fwd_fp8(d["q"], kc8, d["block_table"], d["seqlens"], x.scale, x.causal,
-                               meta, ns, ws, out, lse)
-
-    for _ in range(max(warmup, 3)):
-        flush.zero_()
-        call()
-    torch.cuda.synchronize()
-    ts = []
-    for _ in range(steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        call()
-        b.record(stream)
-        b.synchronize()
-        ts.append(a.elapsed_time(b) * 1e3)
+    # timed like the bf16 decode call: graph replays of the call alone (the schedule is
+    # the metadata call's, the same for both formats)
+    timer = StepTimer(
+        lambda: mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns),
+        lambda: mla.mla_decode_fwd_fp8(d["q"], kc8, d["block_table"], d["seqlens"], x.scale,
+                                       x.causal, meta, ns, ws, out, lse),
+        warmup, flush, stream, False)
+    ts = [t * 1e3 for t in timer.time("decode", steps)]
+    timer.release()
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the FP8 decode: {mla.status_string(st)} {word:#x}")
@@ -472,7 +502,8 @@ def time_fp8(mla, seed, flush, stream, steps, warmup, hbm_peak):
             "us_per_call": us, "GB/s": gbs, "hbm_frac": gbs / hbm_peak,
             "algorithmic_bytes": nbytes,
             "bf16_cache_bytes_same_workload": tokens * 1152 + rows_total * (1152 + 1024 + 4),
-            "note": "mla_decode_fwd_fp8 per call, L2 flushed (256 MB write) before each: "
+            "note": "mla_decode_fwd_fp8 alone (graph replays, as the decode call of every "
+                    "workload), L2 flushed (256 MB write) before each: "
                     "its reads are under twice L2 (compare the uniform entry's "
                     "l2_write_flush figure); the cache was quantized on the GPU by "
                     "mla_kv_append_fp8"}
@@ -512,10 +543,11 @@ def main():
     nbytes, nflops = wl.algorithmic_work(x.seqlens, x.s_q, x.h_q, x.causal)
 
     no_flush = flush_free(nbytes)
-    parts = [lambda: mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns),
-             lambda: mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"],
-                                        x.scale, x.causal, meta, ns, ws, out, lse)]
-    time_steps(parts, max(args.warmup, 3), flush, stream, no_flush)
+    timer = StepTimer(
+        lambda: mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns),
+        lambda: mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"],
+                                   x.scale, x.causal, meta, ns, ws, out, lse),
+        args.warmup, flush, stream, no_flush)
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error during warm-up: {mla.status_string(st)} {word:#x}")
@@ -524,15 +556,18 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        meta_ms, decode_ms = time_steps(parts, args.steps, flush, stream, no_flush)
+        step_ms = timer.time("step", args.steps)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    step_ms = [a + b for a, b in zip(meta_ms, decode_ms)]
     total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
-    # the same steps with a 256 MB L2 write before each (every rank, in the same order)
-    fl_meta_ms, fl_decode_ms = (time_steps(parts, args.steps, flush, stream, False)
-                                if no_flush else (meta_ms, decode_ms))
+    # the decode call and the metadata call alone, and the steps with a 256 MB L2 write
+    # before each (every rank, in the same order)
+    decode_ms = timer.time("decode", args.steps)
+    meta_ms = timer.time("metadata", args.steps)
+    fl = ({w: timer.time(w, args.steps, no_flush=False) for w in ("step", "decode")}
+          if no_flush else {"step": step_ms, "decode": decode_ms})
+    timer.release()
     st, word = mla.mla_get_last_device_error()
     if st != 0:
         raise RuntimeError(f"device error during timing: {mla.status_string(st)} {word:#x}")
@@ -697,13 +732,14 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 q and cache; seeded lengths and page permutation)",
             "config": dict(workload_config(x, args.workload),
-                           l2=l2_note(nbytes, no_flush), parallelism=f"replicas x{world}"),
+                           l2=l2_note(nbytes, no_flush), parallelism=f"replicas x{world}",
+                           timing=TIMING_NOTE),
             "tflops": nflops * args.steps * world / (total_ms / 1e3) / 1e12,
             "us_per_call": statistics.median(step_ms) * 1e3,
             "us_per_call_decode": statistics.median(decode_ms) * 1e3,
             "us_per_call_metadata": statistics.median(meta_ms) * 1e3,
             "roofline": roof,
-            "l2_write_flush": flushed_entry(nbytes, fl_meta_ms, fl_decode_ms, hbm_peak),
+            "l2_write_flush": flushed_entry(nbytes, fl["step"], fl["decode"], hbm_peak),
             "e2e": {"value": nbytes * args.steps * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / args.steps,

@@ -338,3 +338,45 @@ def test_bounded_wait_gives_up_and_reports_a_timeout(h_q):
     assert word & 0xFF == 1                          # the timeout kind
     out, lse = run(x, d)
     compare(out, lse, *oracle_all(x), what="after a timeout")
+
+
+@pytest.mark.parametrize("h_q", [128, 16])
+def test_graph_captured_step_follows_new_lengths(h_q):
+    """The step (metadata + decode) captured once as a CUDA graph, as the benchmark and a
+    serving loop replay it: after new lengths are written into the same buffer, a replay
+    schedules and decodes them (the schedule is computed on the device, so nothing of the
+    first lengths is baked into the graph)."""
+    mla = _mla()
+    lens_a = [3000, 17, 900, 64, 1]
+    lens_b = [1500, 9, 899, 1, 1]               # within each row's pages of lens_a
+    x = wl.make_paged_inputs(lens_a, 1, h_q, seed=21, spare_blocks=2, poison=True)
+    d = to_dev(x)
+    nsm = mla.default_num_sms()
+    meta = torch.empty(mla.mla_metadata_ints(nsm), dtype=torch.int32, device="cuda")
+    ns = torch.empty(mla.mla_num_splits_len(x.batch, h_q, 1), dtype=torch.int32, device="cuda")
+    ws = torch.empty(mla.mla_workspace_bytes(x.batch, h_q, 1, nsm), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((x.batch, 1, h_q, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((x.batch, h_q, 1), dtype=torch.float32, device="cuda")
+
+    def step():
+        mla.mla_get_metadata(d["seqlens"], h_q, 1, nsm, meta, ns)
+        mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
+                           x.causal, meta, ns, ws, out, lse)
+
+    step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for lens in (lens_a, lens_b, lens_a):
+        sl = torch.tensor(lens, dtype=torch.int32)
+        d["seqlens"].copy_(sl)
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        st, word = mla.mla_get_last_device_error()
+        assert st == 0, f"device error {mla.status_string(st)} word={word:#x}"
+        ref = oracle.decode(x.q, x.kcache, x.block_table, sl, x.scale, x.causal)
+        compare(out, lse, *ref, what=f"graph replay h_q={h_q} lens={lens}")
+    del g
