@@ -18,6 +18,20 @@ constexpr float kLn2 = 0.6931471805599453f;
 // error recorded since the last read sticks.
 enum ErrorKind : uint32_t { kErrNone = 0, kErrTimeout = 1, kErrBadInput = 2, kErrWorkspace = 3 };
 
+// Programmatic dependent launch. The split kernels are launched with programmatic stream
+// serialization, so they may be scheduled while the metadata kernel before them in the
+// stream still runs (it signals launch_dependents() as it starts): their set-up (barrier
+// initialisation, TMEM allocation, tensor-map prefetch) overlaps it, and each thread then
+// waits in grid_dependency_wait(), before its first global memory access, until the
+// previous kernel has completed and its writes are visible. (The same link from the split
+// kernel to the combine measured slower and is not used.)
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Combine counters per work sequence in the workspace: one per 8-row group of a tile.
 constexpr int kCombineCounters = 16;
 

@@ -836,6 +836,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
     ptx::cluster_sync();            // peer barriers initialised before any remote access
     ptx::tc_fence_after();
     const uint32_t tmem = *sh.tmem_slot();
+    grid_dependency_wait();         // the schedule is written
 
     if (warp < kWarpProducer) {
         run_softmax(p, sh, tmem, crank, warp, lane);

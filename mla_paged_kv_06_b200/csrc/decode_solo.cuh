@@ -882,6 +882,7 @@ decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_page,
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *sh.tmem_slot();
+    grid_dependency_wait();      // the schedule is written
 
     if (warp < 4) {
         run_rows<C>(p, sh, tmem);

@@ -55,6 +55,7 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
                 int32_t* __restrict__ metadata, int32_t* __restrict__ num_splits) {
     __shared__ int64_t warp_sums[33];
     extern __shared__ int32_t dyn[];
+    launch_dependents();         // the decode kernel may set up meanwhile; it waits for us
     const int V = batch * tiles;
     const int overhead = overhead_pages(h_q, s_q);
     int32_t* Cs = in_smem ? dyn : num_splits;               // cumulative costs C[0..V]

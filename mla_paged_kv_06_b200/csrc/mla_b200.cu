@@ -321,6 +321,25 @@ void* noalloc_scratch(int dev) {
     return addr[dev];
 }
 
+// Launches `kernel` with programmatic stream serialization: it may be scheduled before
+// the previous kernel in the stream ends (once that kernel's blocks have all signalled
+// launch_dependents) and waits for it in grid_dependency_wait().
+template <class... KArgs, class... Args>
+cudaError_t launch_programmatic(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                cudaStream_t s, Args&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 mla_status launch_combine(const DecodeParams& p, cudaStream_t s) {
     // one warp per row of a tile; a tile of a sequence with fewer rows needs fewer CTAs
     const int tile_rows = p.rows < kTileRows ? p.rows : kTileRows;
@@ -342,8 +361,9 @@ mla_status launch_solo(const DecodeParams& p, const void* q, const void* kcache,
     if (!make_page_map(&tm_page, kcache, num_blocks, 9) ||
         !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
         return MLA_ERR_CUDA;
-    solo::decode_kernel<C><<<ctas, C::kBlockThreads, C::kSmemAlloc, s>>>(p, tm_page, tm_page, tm_page, tm_q);
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return launch_programmatic(solo::decode_kernel<C>, dim3(ctas), dim3(C::kBlockThreads),
+                               C::kSmemAlloc, s, p, tm_page, tm_page, tm_page, tm_q) == cudaSuccess
+               ? MLA_OK : MLA_ERR_CUDA;
 }
 
 // FP8 cache ([num_blocks][64][656] bytes, rows of MLA_FP8_ROW_BYTES), three views a page
@@ -400,9 +420,9 @@ mla_status launch_solo_f8(const DecodeParams& p, const void* q, const void* kc8,
     if (!make_f8_maps(&tm_codes, &tm_scales, &tm_rope, kc8, num_blocks) ||
         !make_q_map(&tm_q, q, (size_t)p.batch * p.rows, 9, kN))
         return MLA_ERR_CUDA;
-    solo::decode_kernel<C><<<ctas, C::kBlockThreads, C::kSmemAlloc, s>>>(p, tm_codes, tm_scales, tm_rope,
-                                                                       tm_q);
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return launch_programmatic(solo::decode_kernel<C>, dim3(ctas), dim3(C::kBlockThreads),
+                               C::kSmemAlloc, s, p, tm_codes, tm_scales, tm_rope, tm_q) == cudaSuccess
+               ? MLA_OK : MLA_ERR_CUDA;
 }
 
 // The split kernel for these shapes (1-CTA up to 64 rows per sequence, else 2-CTA
@@ -427,9 +447,9 @@ mla_status launch_decode(const DecodeParams& p, const void* q, const void* kcach
             !make_page_map(&tm_pair, kcache, num_blocks, 2) ||
             !make_q_map(&tm_q4, q, q_rows, 4) || !make_q_map(&tm_q5, q, q_rows, 5))
             return MLA_ERR_CUDA;
-        pair::decode_kernel<<<2 * pairs, pair::kThreads, pair::kSmemAlloc, s>>>(p, tm_page, tm_pair,
-                                                                              tm_q4, tm_q5);
-        st = cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+        st = launch_programmatic(pair::decode_kernel, dim3(2 * pairs), dim3(pair::kThreads),
+                                 pair::kSmemAlloc, s, p, tm_page, tm_pair, tm_q4, tm_q5) == cudaSuccess
+                 ? MLA_OK : MLA_ERR_CUDA;
     }
     if (st != MLA_OK) return st;
     return launch_combine(p, s);
