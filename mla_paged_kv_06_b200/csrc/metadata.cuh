@@ -93,33 +93,50 @@ metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q
     }
     __syncthreads();
     auto C = [&](int v) { return (int64_t)Cs[v]; };
-    const int64_t W = header_unit_cost(num_units, tiles, batch, V, C);
-
-    // Phase 2: one thread per unit locates its first and one-past-last page.
-    for (int u = threadIdx.x; u < num_units; u += blockDim.x) {
-        int vb, kb, ve, ke, chunk;
-        unit_range(u, num_units, tiles, batch, V, overhead, C, pages, &vb, &kb, &ve, &ke, &chunk);
-        int32_t* m = metadata + kMetaInts * (u + 1);
-        m[0] = vb; m[1] = kb; m[2] = ve; m[3] = ke; m[4] = chunk;
-        m[5] = 0; m[6] = 0; m[7] = 0;
-    }
-    if (threadIdx.x == 0) {
+    // the header, from a thread that has no unit or sequence of its own when there is one
+    if (threadIdx.x == blockDim.x - 1) {
+        const int64_t W = header_unit_cost(num_units, tiles, batch, V, C);
         metadata[0] = num_units; metadata[1] = tiles; metadata[2] = batch;
         metadata[3] = h_q; metadata[4] = s_q;
         metadata[5] = (int32_t)(W > 0x7fffffffLL ? 0x7fffffff : W);
         metadata[6] = overhead; metadata[7] = tile_aligned(tiles, num_units) ? 1 : 0;
     }
-    __syncthreads();
-
-    // Phase 3: chunk counts -> exclusive prefix into num_splits (over the costs, tile by
-    // tile, when they were kept there).
+    // Phase 2: unit u locates its first and one-past-last page.
+    auto write_unit = [&](int u) {
+        int vb, kb, ve, ke, chunk;
+        unit_range(u, num_units, tiles, batch, V, overhead, C, pages, &vb, &kb, &ve, &ke, &chunk);
+        int32_t* m = metadata + kMetaInts * (u + 1);
+        m[0] = vb; m[1] = kb; m[2] = ve; m[3] = ke; m[4] = chunk;
+        m[5] = 0; m[6] = 0; m[7] = 0;
+    };
+    // Phase 3: chunk counts -> exclusive prefix into num_splits. With the costs in shared
+    // memory the two phases share one pass, a thread taking unit i and sequence i (their
+    // chains overlap, and no barrier separates them); with the costs kept in num_splits,
+    // which phase 3 overwrites, phase 2 runs first and phase 3 goes tile by tile.
+    // A sequence's chunk count reads its own cost C[v] (overwritten only after it is read,
+    // in the same pass), and the costs at multiples of batch: the start C[t batch] of its
+    // tile's line and C[batch] or C[V] for the line's unit cost. The tiles' lines repeat the
+    // same costs, so C[t batch] = t C[batch]: phase 3 takes those from C[batch], read
+    // before the first overwrite.
+    int64_t c_batch = 0;
+    if (!in_smem) {
+        for (int u = threadIdx.x; u < num_units; u += blockDim.x) write_unit(u);
+        c_batch = C(batch);
+        __syncthreads();
+    }
+    auto C3 = [&](int v) {
+        if (in_smem || v % batch != 0) return (int64_t)Cs[v];
+        return (int64_t)(v / batch) * c_batch;
+    };
+    const int span = in_smem && num_units > V ? num_units : V;
     carry = 0;
-    for (int base = 0; base < V; base += blockDim.x) {
-        int v = base + threadIdx.x;
-        int n = v < V ? chunks_of_v(v, num_units, tiles, batch, V, overhead, C, pages) : 0;
+    for (int base = 0; base < span; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        if (in_smem && i < num_units) write_unit(i);
+        int n = i < V ? chunks_of_v(i, num_units, tiles, batch, V, overhead, C3, pages) : 0;
         int64_t pre;
         int64_t tot = block_exclusive_scan(n, warp_sums, &pre);   // also a barrier
-        if (v < V) num_splits[v] = (int32_t)(carry + pre);
+        if (i < V) num_splits[i] = (int32_t)(carry + pre);
         carry += tot;
         __syncthreads();
     }

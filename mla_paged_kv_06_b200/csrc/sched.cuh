@@ -57,21 +57,31 @@ constexpr int kMetaInts = 8;
 // cutting work finer than a few pages loses more than it balances.
 constexpr int kMinUnitCost = 4;
 
+// a / b for a >= 0, b > 0. The values divided here are positions on a cost line of int32
+// costs, so on the device they nearly always fit the 32-bit divide, which is several
+// times shorter than the 64-bit one; the quotient is the same either way.
+MLA_HD int64_t div_nonneg(int64_t a, int64_t b) {
+#ifdef __CUDA_ARCH__
+    if ((((uint64_t)a | (uint64_t)b) >> 32) == 0) return (int64_t)((uint32_t)a / (uint32_t)b);
+#endif
+    return a / b;
+}
+
 // Per-unit cost budget W for a total cost over `units` units.
 MLA_HD int64_t unit_cost(int64_t total, int units) {
-    int64_t w = (total + units - 1) / units;
+    int64_t w = div_nonneg(total + units - 1, units);
     return w < kMinUnitCost ? kMinUnitCost : w;
 }
 
 MLA_HD int ceil_div(int a, int b) { return (a + b - 1) / b; }
-MLA_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+MLA_HD int64_t ceil_div64(int64_t a, int64_t b) { return div_nonneg(a + b - 1, b); }
 
 MLA_HD int num_tiles(int h_q, int s_q) { return ceil_div(h_q * s_q, kTileRows); }
 
 MLA_HD int pages_of(int seqlen) { return seqlen <= 0 ? 0 : ceil_div(seqlen, kBlock); }
 
 // Unit owning cost position p.
-MLA_HD int unit_of(int64_t p, int64_t W) { return (int)(p / W); }
+MLA_HD int unit_of(int64_t p, int64_t W) { return (int)div_nonneg(p, W); }
 
 // Chunks work sequence v is split into, from its cost start C[v] and page count.
 MLA_HD int chunks_of(int64_t Cv, int nblk, int64_t W, int overhead) {
@@ -83,7 +93,7 @@ MLA_HD int chunks_of(int64_t Cv, int nblk, int64_t W, int overhead) {
 
 MLA_HD bool tile_aligned(int tiles, int units) { return tiles > 1 && units >= tiles; }
 MLA_HD int tile_first_unit(int t, int tiles, int units) {
-    return (int)(((int64_t)t * units) / tiles);
+    return (int)div_nonneg((int64_t)t * units, tiles);
 }
 
 // Where unit u cuts: the line it cuts (its first work sequence v0 and sequence count n,
@@ -102,7 +112,7 @@ MLA_HD UnitCut cut_of_unit(int u, int units, int tiles, int batch, int V, CostFn
         c.W = unit_cost(C(V), units);
         return c;
     }
-    const int t = (int)((((int64_t)u + 1) * tiles - 1) / units);
+    const int t = (int)div_nonneg(((int64_t)u + 1) * tiles - 1, units);
     const int first = tile_first_unit(t, tiles, units);
     c.v0 = t * batch; c.n = batch; c.local = u - first;
     c.W = unit_cost(C(batch), tile_first_unit(t + 1, tiles, units) - first);
@@ -122,20 +132,31 @@ struct UnitRange {
     int v_begin, page_begin, v_end, page_end, chunk_begin;
 };
 
-// First page position >= target, as (v, page). C(v) returns the cumulative cost
-// C[v] (v in [0, V]) and nblk(v) the page count of v. Returns (V, 0) when no page lies
-// at or after target.
-template <class CostFn, class PagesFn>
-MLA_HD void locate(const int64_t target, CostFn C, PagesFn nblk, int V, int overhead,
-                   int* v_out, int* k_out) {
-    // smallest v with C[v+1] > target: its page range [C[v]+overhead, C[v+1]) ends
-    // after target
-    int lo = 0, hi = V;
-    while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if ((int64_t)C(mid + 1) > target) hi = mid; else lo = mid + 1;
+// Count of i in [1, n] with C(i) <= target, for the two targets t0 <= t1 at once (two
+// independent load chains per step). C is non-decreasing with C(0) = 0 <= t0, so this is
+// the smallest v with C(v + 1) > target, or n when there is none.
+template <class CostFn>
+MLA_HD void count_le_pair(int64_t t0, int64_t t1, CostFn C, int n, int* c0, int* c1) {
+    int step = 1;
+    while (step * 2 <= n) step *= 2;
+    int a = 0, b = 0;
+    for (; n > 0 && step > 0; step >>= 1) {
+        const bool ina = a + step <= n, inb = b + step <= n;
+        const int64_t ca = ina ? (int64_t)C(a + step) : 0;
+        const int64_t cb = inb ? (int64_t)C(b + step) : 0;
+        if (ina && ca <= t0) a += step;
+        if (inb && cb <= t1) b += step;
     }
-    int v = lo;
+    *c0 = a;
+    *c1 = b;
+}
+
+// First page position >= target, as (v, page), given v = the smallest work sequence
+// whose range [C[v] + overhead, C[v + 1]) ends after target (count_le_pair). Returns
+// (V, 0) when no page lies at or after target.
+template <class CostFn, class PagesFn>
+MLA_HD void locate_from(int v, const int64_t target, CostFn C, PagesFn nblk, int V,
+                        int overhead, int* v_out, int* k_out) {
     while (v < V && nblk(v) == 0) ++v;     // empty sequences own no page
     if (v >= V) { *v_out = V; *k_out = 0; return; }
     int64_t k = target - ((int64_t)C(v) + overhead);
@@ -152,9 +173,11 @@ MLA_HD void unit_range(int u, int units, int tiles, int batch, int V, int overhe
     const int64_t base = C(c.v0);
     auto Cl = [&](int i) { return (int64_t)C(c.v0 + i) - base; };
     auto Pl = [&](int i) { return nblk(c.v0 + i); };
+    const int64_t t0 = (int64_t)c.local * c.W, t1 = t0 + c.W;
     int b0, k0, b1, k1;
-    locate((int64_t)c.local * c.W, Cl, Pl, c.n, overhead, &b0, &k0);
-    locate((int64_t)(c.local + 1) * c.W, Cl, Pl, c.n, overhead, &b1, &k1);
+    count_le_pair(t0, t1, Cl, c.n, &b0, &b1);
+    locate_from(b0, t0, Cl, Pl, c.n, overhead, &b0, &k0);
+    locate_from(b1, t1, Cl, Pl, c.n, overhead, &b1, &k1);
     int ch = 0;
     if (b0 < c.n && (b0 != b1 || k0 != k1)) ch = c.local - unit_of(Cl(b0) + overhead, c.W);
     *vb = c.v0 + b0; *kb = k0; *ve = c.v0 + b1; *ke = k1; *chunk = ch;

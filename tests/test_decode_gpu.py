@@ -125,10 +125,12 @@ def test_small_parity(case, num_sms, impl):
 
 def test_device_metadata_matches_host_plan():
     mla = _mla()
-    # the last case is too large for the scheduler's shared-memory table (global path)
+    # the last two cases are too large for the scheduler's shared-memory table (global
+    # path); the last one has two row tiles per sequence, cut tile by tile
     for lens, h_q, s_q in [([37, 130], 16, 1), ([65536, 10, 0, 65536, 3], 64, 1),
                            ([8192] * 128, 128, 2), (list(range(0, 9000, 37)), 128, 1),
-                           ([5, 700, 0, 64] * 7500, 16, 1)]:
+                           ([5, 700, 0, 64] * 7500, 16, 1),
+                           ([5, 700, 0, 64, 3000] * 4200, 128, 2)]:
         seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
         for nsm in [1, 2, 13, mla.default_num_sms()]:
             meta, ns = mla.mla_get_metadata(seq, h_q, s_q, nsm)
