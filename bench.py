@@ -787,7 +787,7 @@ def main():
 
 
 # Bumped whenever the split kernel changes, so stale ncu traffic is never reported.
-KERNEL_REV = "pair-6"
+KERNEL_REV = "pair-7"
 
 if __name__ == "__main__":
     sys.exit(main())
