@@ -34,6 +34,11 @@
  * (a cudaStream_t passed as void*; NULL is the legacy default stream) and never
  * synchronise it. The first mla_decode_fwd on a device also sets the kernel's
  * shared-memory limit and queries its cluster occupancy once (cached afterwards).
+ * The decode calls launch their split kernel with programmatic stream serialization
+ * (CUDA's programmatic dependent launch): it may be scheduled while the kernel before
+ * it on `stream` (normally mla_get_metadata's) still runs, but it reads and writes no
+ * global memory before that kernel has completed, so stream order holds as for any
+ * launch. The calls can be captured into a CUDA graph.
  *
  * Errors: every call checks its arguments on the host first and returns a negative
  * mla_status without launching anything when they are invalid. A launch failure is
