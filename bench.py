@@ -334,7 +334,9 @@ def capture(parts):
     ABI are recorded once and replayed as one unit, as a serving loop replays its step)."""
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
+    # thread-local capture: under torchrun the process group's watchdog thread keeps
+    # querying its events, which a global-mode capture would refuse
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
         for f in parts:
             f()
     torch.cuda.synchronize()
