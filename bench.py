@@ -444,6 +444,7 @@ def time_config(mla, name, seed, flush, stream, steps, warmup, hbm_peak, tf_peak
              "s_q": x.s_q, "h_q": x.h_q, "total_tokens": int(x.seqlens.sum()),
              "kernel": "1-CTA (rows <= 64)" if rows <= 64 else "2-CTA pairs",
              "l2": l2_note(nbytes, no_flush),
+             "work_units": mla.mla_num_work_units(nsm, x.h_q, x.s_q),
              "us_per_call": statistics.median(step_ms) * 1e3,
              "us_per_call_decode": statistics.median(decode_ms) * 1e3,
              "us_per_call_metadata": statistics.median(meta_ms) * 1e3,
@@ -740,6 +741,9 @@ def main():
             "us_per_call": statistics.median(step_ms) * 1e3,
             "us_per_call_decode": statistics.median(decode_ms) * 1e3,
             "us_per_call_metadata": statistics.median(meta_ms) * 1e3,
+            # 2-CTA clusters (more than 64 query rows) or CTAs the chip runs at once: the
+            # clusters a chip fits vary with its SM layout, and the 2-CTA kernel's time with them
+            "work_units": mla.mla_num_work_units(nsm, x.h_q, x.s_q),
             "roofline": roof,
             "l2_write_flush": flushed_entry(nbytes, fl["step"], fl["decode"], hbm_peak),
             "e2e": {"value": nbytes * args.steps * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
@@ -768,7 +772,7 @@ def main():
         main_entry = {"workload": line["config"]["workload"], "batch": x.batch, "s_q": x.s_q,
                       "h_q": x.h_q, "total_tokens": int(x.seqlens.sum()),
                       "kernel": "1-CTA (rows <= 64)" if x.s_q * x.h_q <= 64 else "2-CTA pairs",
-                      "l2": line["config"]["l2"],
+                      "l2": line["config"]["l2"], "work_units": line["work_units"],
                       "us_per_call": line["us_per_call"],
                       "us_per_call_decode": line["us_per_call_decode"],
                       "us_per_call_metadata": line["us_per_call_metadata"],
