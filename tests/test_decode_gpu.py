@@ -58,6 +58,37 @@ def run(x, d=None, impl="tc", num_sms=None, check_error=True):
     return out, lse
 
 
+def graph_step(x, d):
+    """The step as the benchmark times it: mla_get_metadata + mla_decode_fwd captured once
+    as a CUDA graph on buffers of their own, then replayed."""
+    mla = _mla()
+    nsm = mla.default_num_sms()
+    meta = torch.empty(mla.mla_metadata_ints(nsm), dtype=torch.int32, device="cuda")
+    ns = torch.empty(mla.mla_num_splits_len(x.batch, x.h_q, x.s_q), dtype=torch.int32,
+                     device="cuda")
+    ws = torch.empty(mla.mla_workspace_bytes(x.batch, x.h_q, x.s_q, nsm), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.full((x.batch, x.s_q, x.h_q, 512), float("nan"), dtype=torch.bfloat16,
+                     device="cuda")
+    lse = torch.empty((x.batch, x.h_q, x.s_q), dtype=torch.float32, device="cuda")
+
+    def step():
+        mla.mla_get_metadata(d["seqlens"], x.h_q, x.s_q, nsm, meta, ns)
+        mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
+                           x.causal, meta, ns, ws, out, lse)
+
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    g.replay()
+    torch.cuda.synchronize()
+    st, word = mla.mla_get_last_device_error()
+    assert st == 0, f"device error {mla.status_string(st)} word={word:#x}"
+    del g
+    return out, lse
+
+
 def compare(out, lse, ref_out, ref_lse, what=""):
     o = out.double().cpu().numpy()
     l = lse.double().cpu().numpy()
@@ -244,6 +275,9 @@ def test_full_workload_parity(name, full_inputs):
     ref_out, ref_lse = oracle_all(x)
     d_o, d_l, rel = compare(out, lse, ref_out, ref_lse, what=name)
     print(f"{name}: max|dout| {d_o:.3e}  max|dlse| {d_l:.3e}  max row-relative {rel:.3e}")
+    # the benchmark replays the step as a CUDA graph: the replay gives the same bits
+    g_out, g_lse = graph_step(x, d)
+    assert torch.equal(g_out, out) and torch.equal(g_lse, lse), f"{name}: graph replay differs"
 
 
 @pytest.mark.parametrize("name", FULL)
