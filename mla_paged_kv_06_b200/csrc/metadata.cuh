@@ -44,11 +44,11 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t* smem
 // metadata: header {num_units, tiles, batch, h_q, s_q, unit_cost, overhead, tile_aligned}
 // then one
 // {v_begin, page_begin, v_end, page_end, chunk_begin, 0, 0, 0} per unit.
-// num_splits holds the cumulative costs C[v] while the units are located, then is
-// overwritten with the chunk prefix.
-// `in_smem`: the cost table and page counts live in dynamic shared memory (the launch
-// provides (V + 1 + batch) int32), so the per-unit binary searches never wait on L2;
-// otherwise the costs are kept in num_splits and the lengths re-read from seqlens.
+// `in_smem`: the cost table C[0..V] and page counts live in dynamic shared memory (the
+// launch provides (V + 1 + batch) int32), so the per-unit searches never wait on L2, and
+// one pass locates the units and counts the chunks; otherwise num_splits holds the costs
+// while the units are located, is then overwritten with the chunk prefix, and the lengths
+// are re-read from seqlens.
 __global__ void __launch_bounds__(kMetaThreads)
 metadata_kernel(const int32_t* __restrict__ seqlens, int batch, int h_q, int s_q, int tiles,
                 int num_units, int in_smem,
