@@ -416,3 +416,28 @@ def test_graph_captured_step_follows_new_lengths(h_q):
         ref = oracle.decode(x.q, x.kcache, x.block_table, sl, x.scale, x.causal)
         compare(out, lse, *ref, what=f"graph replay h_q={h_q} lens={lens}")
     del g
+
+
+@pytest.mark.parametrize("h_q", [128, 16])
+def test_decode_sees_the_writes_of_the_kernel_queued_before_it(h_q):
+    """The split kernel is launched with programmatic stream serialization: it may be
+    scheduled before the kernel ahead of it ends, and must still read only what that
+    kernel wrote. Here a torch kernel rewrites q in place right before the decode, with no
+    synchronisation, and the decode must see the new q (it then matches the oracle on it)."""
+    mla = _mla()
+    x = wl.make_paged_inputs([1500, 64, 700, 1], 1, h_q, seed=31, spare_blocks=2, poison=True)
+    d = to_dev(x)
+    nsm = mla.default_num_sms()
+    meta, ns = mla.mla_get_metadata(d["seqlens"], h_q, 1, nsm)
+    mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"], x.scale,
+                       x.causal, meta, ns, num_sms=nsm)
+    d["q"].mul_(-1.5)                          # queued right before the decode
+    out, lse = mla.mla_decode_fwd(d["q"], d["kcache"], d["block_table"], d["seqlens"],
+                                  x.scale, x.causal, meta, ns, num_sms=nsm)
+    torch.cuda.synchronize()
+    st, word = mla.mla_get_last_device_error()
+    assert st == 0, f"device error {mla.status_string(st)} word={word:#x}"
+    q_new = d["q"].cpu()
+    assert torch.equal(q_new, (x.q.cuda() * -1.5).cpu())
+    ref = oracle.decode(q_new, x.kcache, x.block_table, x.seqlens, x.scale, x.causal)
+    compare(out, lse, *ref, what=f"q rewritten before the decode, h_q={h_q}")
